@@ -1,0 +1,210 @@
+/*
+ * CPU oracle for the CSA lightning-indexer top-k step.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the
+ * benchmark's CPU-baseline leg may load or call this file.  It shares no code,
+ * header, table or helper with the CUDA library, and the library never calls
+ * it.
+ *
+ * What it computes (StreamIndex, "Memory-Bounded Compressed Sparse Attention
+ * via Streaming Top-k", abstract: a lightning indexer -- a learned scoring
+ * projection over compressed keys -- scores the compressed keys and the top-k
+ * are selected per query).  The scoring function is the DeepSeek-V3.2
+ * lightning-indexer form, which the pages name only as that lineage:
+ *
+ *     I[b,t,s] = sum_h w[b,t,h] * ReLU( sum_d q[b,t,h,d] * kc[b,s,d] )
+ *
+ * Compressed key s covers tokens [s*m, s*m+m-1]; it is visible to query t iff
+ * s*m+m-1 <= t (and s < T), so row t sees n(t) = min(T, floor((t+1)/m))
+ * keys, namely s = 0..n(t)-1.  The row's result is its visible keys fully
+ * sorted by (score descending, index ascending), truncated to k, padded with
+ * index -1 / score -inf when n(t) < k.
+ *
+ * Arithmetic: every input value is widened exactly to double (bf16 -> double
+ * is exact; e4m3 -> double is exact; scales and w are fp32, exact in double),
+ * dot products are summed in d order, heads in h order, all in double.  The
+ * reported score is the double result rounded to float.  Plain loops,
+ * single-threaded, no SIMD intrinsics; qsort for the full sort.
+ *
+ * Parity pins (tests): hand-worked 4x4 cases, the matmul special cases, the
+ * visible-pair closed form, the causal invariant, prefix monotonicity of
+ * top-k, brute force over all k-subsets, head-permutation and power-of-two
+ * scaling invariances, integer-exact inputs.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* bf16 bit pattern -> double (bf16 is the top half of an IEEE binary32). */
+double oracle_bf16_value(uint16_t bits) {
+  uint32_t u = (uint32_t)bits << 16;
+  float f;
+  memcpy(&f, &u, 4);
+  return (double)f;
+}
+
+/* OCP FP8 E4M3: sign, 4 exponent bits (bias 7), 3 mantissa bits; exponent
+ * field 0 is subnormal (m * 2^-9); S.1111.111 is NaN; no infinities. */
+double oracle_e4m3_value(uint8_t bits) {
+  int sign = bits >> 7, e = (bits >> 3) & 15, m = bits & 7;
+  double v;
+  if (e == 15 && m == 7) return NAN;
+  if (e == 0) v = ldexp((double)m, -9);
+  else v = ldexp(1.0 + m / 8.0, e - 7);
+  return sign ? -v : v;
+}
+
+/* Number of keys visible to query t: key s is visible iff s*m+m-1 <= t. */
+int64_t oracle_visible_count(int64_t t, int64_t T, int64_t m) {
+  int64_t n = (t + 1) / m;
+  return n < T ? n : T;
+}
+
+/* One indexer score in double from already-widened rows.
+ * qT: D*H (d-major, i.e. the query row transposed), krow: D, wrow: H,
+ * dot: H doubles of scratch.  Each head's dot product is summed over d in
+ * increasing order; the loop runs the H independent sums side by side. */
+static double score_rows(const double* qT, const double* krow, const double* wrow, int H, int D,
+                         double* dot) {
+  for (int h = 0; h < H; ++h) dot[h] = 0.0;
+  for (int d = 0; d < D; ++d) {
+    const double kd = krow[d];
+    const double* qd = qT + (size_t)d * H;
+    for (int h = 0; h < H; ++h) dot[h] += qd[h] * kd;
+  }
+  double acc = 0.0;
+  for (int h = 0; h < H; ++h) {
+    double r = dot[h] > 0.0 ? dot[h] : 0.0;
+    acc += wrow[h] * r;
+  }
+  return acc;
+}
+
+typedef struct { double score; int64_t idx; } cand_t;
+
+/* score descending, then index ascending */
+static int cand_cmp(const void* pa, const void* pb) {
+  const cand_t* a = (const cand_t*)pa;
+  const cand_t* b = (const cand_t*)pb;
+  if (a->score > b->score) return -1;
+  if (a->score < b->score) return 1;
+  return (a->idx > b->idx) - (a->idx < b->idx);
+}
+
+/* Widening of one query row / key row / weight row to double. */
+typedef struct {
+  int fmt; /* 0 bf16, 1 e4m3 */
+  const void* q; const float* q_scale;
+  const void* kc; const float* kc_scale;
+  const float* w;
+  int64_t B, S, T, H, D, m;
+} problem_t;
+
+/* qrow receives the query's H x D values transposed to D x H. */
+static void widen_query(const problem_t* p, int64_t b, int64_t t, double* qrow, double* wrow) {
+  int64_t base = (b * p->S + t) * p->H;
+  for (int64_t h = 0; h < p->H; ++h) {
+    wrow[h] = (double)p->w[base + h];
+    for (int64_t d = 0; d < p->D; ++d) {
+      int64_t i = (base + h) * p->D + d;
+      if (p->fmt == 0) qrow[d * p->H + h] = oracle_bf16_value(((const uint16_t*)p->q)[i]);
+      else qrow[d * p->H + h] = oracle_e4m3_value(((const uint8_t*)p->q)[i]) * (double)p->q_scale[base + h];
+    }
+  }
+}
+
+static void widen_key(const problem_t* p, int64_t b, int64_t s, double* krow) {
+  int64_t r = b * p->T + s;
+  for (int64_t d = 0; d < p->D; ++d) {
+    int64_t i = r * p->D + d;
+    if (p->fmt == 0) krow[d] = oracle_bf16_value(((const uint16_t*)p->kc)[i]);
+    else krow[d] = oracle_e4m3_value(((const uint8_t*)p->kc)[i]) * (double)p->kc_scale[r];
+  }
+}
+
+/*
+ * Top-k for the listed rows.  rows[i] = b*S + t.  Outputs are [n_rows, k]:
+ * out_idx (int32, -1 padded), out_score (float, -inf padded, may be NULL),
+ * out_score64 (double, -inf padded, may be NULL).  Returns 0, or -1 on a bad
+ * argument, -2 on allocation failure.
+ */
+static int topk_rows(const problem_t* p, int64_t k, const int64_t* rows, int64_t n_rows,
+                     int32_t* out_idx, float* out_score, double* out_score64) {
+  if (p->B <= 0 || p->S <= 0 || p->T <= 0 || p->H <= 0 || p->D <= 0 || p->m <= 0 || k <= 0) return -1;
+  double* qrow = (double*)malloc(sizeof(double) * (size_t)(p->H * p->D));
+  double* wrow = (double*)malloc(sizeof(double) * (size_t)p->H);
+  double* krow = (double*)malloc(sizeof(double) * (size_t)p->D);
+  double* dot = (double*)malloc(sizeof(double) * (size_t)p->H);
+  cand_t* c = (cand_t*)malloc(sizeof(cand_t) * (size_t)p->T);
+  if (!qrow || !wrow || !krow || !dot || !c) {
+    free(qrow); free(wrow); free(krow); free(dot); free(c);
+    return -2;
+  }
+  for (int64_t i = 0; i < n_rows; ++i) {
+    int64_t r = rows[i];
+    if (r < 0 || r >= p->B * p->S) { free(qrow); free(wrow); free(krow); free(dot); free(c); return -1; }
+    int64_t b = r / p->S, t = r % p->S;
+    int64_t n = oracle_visible_count(t, p->T, p->m);
+    widen_query(p, b, t, qrow, wrow);
+    for (int64_t s = 0; s < n; ++s) {
+      widen_key(p, b, s, krow);
+      c[s].score = score_rows(qrow, krow, wrow, (int)p->H, (int)p->D, dot);
+      c[s].idx = s;
+    }
+    qsort(c, (size_t)n, sizeof(cand_t), cand_cmp);
+    for (int64_t j = 0; j < k; ++j) {
+      int64_t o = i * k + j;
+      if (j < n) {
+        out_idx[o] = (int32_t)c[j].idx;
+        if (out_score) out_score[o] = (float)c[j].score;
+        if (out_score64) out_score64[o] = c[j].score;
+      } else {
+        out_idx[o] = -1;
+        if (out_score) out_score[o] = -INFINITY;
+        if (out_score64) out_score64[o] = -INFINITY;
+      }
+    }
+  }
+  free(qrow); free(wrow); free(krow); free(dot); free(c);
+  return 0;
+}
+
+/* bf16 q [B,S,H,D], bf16 kc [B,T,D], fp32 w [B,S,H]. */
+int oracle_topk_bf16(const uint16_t* q, const uint16_t* kc, const float* w, int64_t B, int64_t S,
+                     int64_t T, int64_t H, int64_t D, int64_t m, int64_t k, const int64_t* rows,
+                     int64_t n_rows, int32_t* out_idx, float* out_score, double* out_score64) {
+  problem_t p = {0, q, NULL, kc, NULL, w, B, S, T, H, D, m};
+  return topk_rows(&p, k, rows, n_rows, out_idx, out_score, out_score64);
+}
+
+/* e4m3 q [B,S,H,D] with q_scale [B,S,H]; e4m3 kc [B,T,D] with kc_scale [B,T];
+ * each value dequantised as code value * its row's scale. */
+int oracle_topk_e4m3(const uint8_t* q, const float* q_scale, const uint8_t* kc,
+                     const float* kc_scale, const float* w, int64_t B, int64_t S, int64_t T,
+                     int64_t H, int64_t D, int64_t m, int64_t k, const int64_t* rows,
+                     int64_t n_rows, int32_t* out_idx, float* out_score, double* out_score64) {
+  problem_t p = {1, q, q_scale, kc, kc_scale, w, B, S, T, H, D, m};
+  return topk_rows(&p, k, rows, n_rows, out_idx, out_score, out_score64);
+}
+
+/* All T scores of one row (bf16 inputs) in double; invisible keys get NaN.
+ * For brute-force and invariant tests on small inputs. */
+int oracle_scores_bf16(const uint16_t* q, const uint16_t* kc, const float* w, int64_t B, int64_t S,
+                       int64_t T, int64_t H, int64_t D, int64_t m, int64_t row, double* out) {
+  problem_t p = {0, q, NULL, kc, NULL, w, B, S, T, H, D, m};
+  if (row < 0 || row >= B * S) return -1;
+  double* qrow = (double*)malloc(sizeof(double) * (size_t)(H * D));
+  double* wrow = (double*)malloc(sizeof(double) * (size_t)H);
+  double* krow = (double*)malloc(sizeof(double) * (size_t)D);
+  double* dot = (double*)malloc(sizeof(double) * (size_t)H);
+  if (!qrow || !wrow || !krow || !dot) { free(qrow); free(wrow); free(krow); free(dot); return -2; }
+  int64_t b = row / S, t = row % S, n = oracle_visible_count(t, T, m);
+  widen_query(&p, b, t, qrow, wrow);
+  for (int64_t s = 0; s < T; ++s) {
+    if (s < n) { widen_key(&p, b, s, krow); out[s] = score_rows(qrow, krow, wrow, (int)H, (int)D, dot); }
+    else out[s] = NAN;
+  }
+  free(qrow); free(wrow); free(krow); free(dot);
+  return 0;
+}

@@ -1,0 +1,237 @@
+"""Seeded synthetic inputs for the CSA lightning-indexer top-k step.
+
+Shared by the CUDA path's tests and benchmark and by the CPU oracle's tests.
+Nothing here computes an indexer score or a top-k: it only draws numbers
+(counter-based SplitMix64, Box-Muller normals) and stores them as bf16,
+fp8 e4m3 with per-row fp32 scales, or fp32.  The C source is ``synth.c``;
+it is compiled on first use into ``libsynth.so`` beside it.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from dataclasses import dataclass, field
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "synth.c")
+_LIB = os.path.join(_HERE, "libsynth.so")
+_lib = None
+
+TENSOR_Q, TENSOR_KC, TENSOR_W = 1, 2, 3
+
+
+def build(force: bool = False) -> str:
+    """Compile libsynth.so (gcc, -O2, pthreads) if missing or stale."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.run(["gcc", "-O2", "-std=c11", "-D_GNU_SOURCE", "-shared", "-fPIC", "-pthread",
+                        "-o", tmp, _SRC, "-lm"], check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_LIB)
+        L.synth_draw.restype = ctypes.c_uint64
+        L.synth_draw.argtypes = [ctypes.c_uint64, ctypes.c_uint64]
+        L.synth_stream_key.restype = ctypes.c_uint64
+        L.synth_stream_key.argtypes = [ctypes.c_uint64, ctypes.c_uint32]
+        L.synth_normal.restype = ctypes.c_double
+        L.synth_normal.argtypes = [ctypes.c_uint64, ctypes.c_uint64]
+        L.synth_f32_to_bf16.restype = ctypes.c_uint16
+        L.synth_f32_to_bf16.argtypes = [ctypes.c_float]
+        L.synth_f32_to_e4m3.restype = ctypes.c_uint8
+        L.synth_f32_to_e4m3.argtypes = [ctypes.c_float]
+        L.synth_matrix.restype = ctypes.c_int
+        L.synth_matrix.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
+                                   ctypes.c_uint64, ctypes.c_uint32, ctypes.c_int, ctypes.c_double,
+                                   ctypes.c_int, ctypes.c_int]
+        L.synth_keys_planted.restype = ctypes.c_int
+        L.synth_keys_planted.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
+                                         ctypes.c_int, ctypes.c_uint64, ctypes.c_uint32, ctypes.c_double,
+                                         ctypes.c_double, ctypes.c_double, ctypes.c_int, ctypes.c_int,
+                                         ctypes.c_void_p]
+        L.synth_weights.restype = ctypes.c_int
+        L.synth_weights.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_uint64, ctypes.c_uint32,
+                                    ctypes.c_int, ctypes.c_double, ctypes.c_int]
+        L.synth_sample_rows.restype = ctypes.c_int
+        L.synth_sample_rows.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                        ctypes.c_uint64]
+        _lib = L
+    return _lib
+
+
+def _threads() -> int:
+    return max(1, min(64, os.cpu_count() or 1))
+
+
+def _ptr(a: np.ndarray) -> int:
+    return a.ctypes.data
+
+
+def matrix(rows: int, D: int, seed: int, tensor_id: int, kind: str = "gauss", sigma: float = 1.0,
+           fmt: str = "bf16", out: np.ndarray | None = None, scale_out: np.ndarray | None = None):
+    """rows x D matrix. kind 'gauss' (N(0,1)*sigma) or 'int' ({-3..3}).
+
+    fmt 'bf16' -> uint16 array of bf16 bit patterns; 'e4m3' -> (uint8 codes,
+    float32 per-row scales)."""
+    k = {"gauss": 0, "int": 1}[kind]
+    if fmt == "bf16":
+        o = out if out is not None else np.empty((rows, D), dtype=np.uint16)
+        rc = lib().synth_matrix(_ptr(o), None, rows, D, seed, tensor_id, k, sigma, 0, _threads())
+        assert rc == 0
+        return o
+    o = out if out is not None else np.empty((rows, D), dtype=np.uint8)
+    s = scale_out if scale_out is not None else np.empty((rows,), dtype=np.float32)
+    rc = lib().synth_matrix(_ptr(o), _ptr(s), rows, D, seed, tensor_id, k, sigma, 1, _threads())
+    assert rc == 0
+    return o, s
+
+
+def keys_planted(B: int, T: int, D: int, seed: int, tensor_id: int, sigma: float, frac: float,
+                 boost: float, fmt: str = "bf16", with_mask: bool = False):
+    """[B*T, D] keys, N(0,1)*sigma with round(frac*T) rows per sequence boosted
+    by `boost` times a per-sequence unit direction."""
+    mask = np.empty((B * T,), dtype=np.uint8) if with_mask else None
+    mptr = _ptr(mask) if with_mask else None
+    if fmt == "bf16":
+        o = np.empty((B * T, D), dtype=np.uint16)
+        rc = lib().synth_keys_planted(_ptr(o), None, B, T, D, seed, tensor_id, sigma, frac, boost, 0,
+                                      _threads(), mptr)
+        assert rc == 0
+        return (o, mask) if with_mask else o
+    o = np.empty((B * T, D), dtype=np.uint8)
+    s = np.empty((B * T,), dtype=np.float32)
+    rc = lib().synth_keys_planted(_ptr(o), _ptr(s), B, T, D, seed, tensor_id, sigma, frac, boost, 1,
+                                  _threads(), mptr)
+    assert rc == 0
+    return ((o, s), mask) if with_mask else (o, s)
+
+
+def weights(n: int, seed: int, tensor_id: int, kind: str = "uniform", scale: float = 1.0,
+            out: np.ndarray | None = None) -> np.ndarray:
+    """n fp32 weights: 'uniform' U(0,1)*scale, or 'pow2' 2^-j with j in {0..6}."""
+    o = out if out is not None else np.empty((n,), dtype=np.float32)
+    rc = lib().synth_weights(_ptr(o), n, seed, tensor_id, {"uniform": 0, "pow2": 1}[kind], scale,
+                             _threads())
+    assert rc == 0
+    return o
+
+
+def sample_rows(count: int, lo: int, hi: int, seed: int) -> np.ndarray:
+    """`count` distinct integers drawn uniformly from [lo, hi), sorted."""
+    o = np.empty((count,), dtype=np.int64)
+    rc = lib().synth_sample_rows(_ptr(o), count, lo, hi, seed)
+    assert rc == 0
+    return o
+
+
+def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
+    """Widen bf16 bit patterns to float32 (exact)."""
+    return (bits.astype(np.uint32) << 16).view(np.float32)
+
+
+def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round float32 to bf16 (nearest-even) bit patterns, vectorised."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    u = u + 0x7FFF + ((u >> 16) & 1)
+    return (u >> 16).astype(np.uint16)
+
+
+# --------------------------------------------------------------------------
+# The indexer workloads.  Shapes and value distributions are the tiny,
+# integer-exact, sweep, V4-Flash and million-token cases of the lightning
+# indexer at compression ratio m=4, H_I=64 heads, D=128.
+# --------------------------------------------------------------------------
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    S: int
+    m: int
+    H: int
+    D: int
+    k: int
+    seed: int
+    kind: str            # "gauss" | "int" | "planted"
+    sweep: dict = field(default_factory=dict, compare=False, hash=False)
+
+    @property
+    def T(self) -> int:
+        return self.S // self.m
+
+    def visible_pairs(self) -> int:
+        """Number of causally visible (query, key) pairs for one sequence."""
+        return self.B * visible_pairs(self.S, self.T, self.m)
+
+
+def visible_pairs(S: int, T: int, m: int) -> int:
+    """sum over t in [0, S) of min(T, floor((t+1)/m)), in closed form.
+
+    With x = t+1: floor(x/m) < T for x <= m*T-1, and the sum of floor(x/m) for
+    x = 1..N is m*q*(q-1)/2 + q*(r+1) with (q, r) = divmod(N, m)."""
+    upto = min(S, m * T - 1)
+    q, r = divmod(upto, m)
+    return m * q * (q - 1) // 2 + q * (r + 1) + (S - upto) * T
+
+
+WORKLOADS = {
+    "tiny": Workload("tiny", 1, 1024, 4, 64, 128, 64, 0, "gauss"),
+    "integer": Workload("integer", 1, 8192, 4, 64, 128, 512, 1, "int"),
+    "sweep": Workload("sweep", 1, 16384, 4, 64, 128, 512, 2, "gauss",
+                      sweep={"query_chunk": [256, 512, 1024, 2048, 4096],
+                             "key_tile": [64, 128, 256, 512, 1024],
+                             "k": [64, 128, 256, 512, 1024]}),
+    "v4flash": Workload("v4flash", 1, 65536, 4, 64, 128, 512, 3, "planted"),
+    "million": Workload("million", 1, 1048576, 4, 64, 128, 512, 4, "planted"),
+}
+
+PLANTED_FRAC = 0.05
+PLANTED_BOOST = 2.0
+
+
+def make_inputs(wl: Workload, fmt: str = "bf16", S: int | None = None, B: int | None = None,
+                seed: int | None = None):
+    """Generate (q, kc, w[, q_scale, kc_scale]) host arrays for a workload.
+
+    q: [B, S, H, D] (bf16 bits uint16, or e4m3 uint8 + q_scale [B, S, H])
+    kc: [B, T, D]   (bf16 bits, or e4m3 + kc_scale [B, T])
+    w: [B, S, H] float32
+    `S`, `B` and `seed` override the workload's (for reduced-size cases).
+    """
+    S = wl.S if S is None else S
+    B = wl.B if B is None else B
+    seed = wl.seed if seed is None else seed
+    T = S // wl.m
+    H, D = wl.H, wl.D
+    sig = 1.0 / np.sqrt(D)
+    kind = "int" if wl.kind == "int" else "gauss"
+    qsig = 1.0 if kind == "int" else sig
+    res = {}
+    if fmt == "bf16":
+        q = matrix(B * S * H, D, seed, TENSOR_Q, kind, qsig, "bf16").reshape(B, S, H, D)
+    else:
+        q8, qs = matrix(B * S * H, D, seed, TENSOR_Q, kind, qsig, "e4m3")
+        q = q8.reshape(B, S, H, D)
+        res["q_scale"] = qs.reshape(B, S, H)
+    if wl.kind == "planted":
+        kcr = keys_planted(B, T, D, seed, TENSOR_KC, sig, PLANTED_FRAC, PLANTED_BOOST, fmt)
+    else:
+        kcr = matrix(B * T, D, seed, TENSOR_KC, kind, qsig, fmt)
+    if fmt == "bf16":
+        kc = kcr.reshape(B, T, D)
+    else:
+        kc = kcr[0].reshape(B, T, D)
+        res["kc_scale"] = kcr[1].reshape(B, T)
+    if wl.kind == "int":
+        w = weights(B * S * H, seed, TENSOR_W, "pow2").reshape(B, S, H)
+    else:
+        w = weights(B * S * H, seed, TENSOR_W, "uniform", 1.0 / np.sqrt(H)).reshape(B, S, H)
+    res.update(q=q, kc=kc, w=w)
+    return res

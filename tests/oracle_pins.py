@@ -1,0 +1,223 @@
+"""Pins for the CPU oracle: checks that do not restate its formula.
+
+Each check takes a ctypes handle on an oracle library, so the same checks run
+on the real oracle (test_oracle_pins.py) and on copies with a planted mistake
+(test_oracle_mutants.py), which must each fail at least one of them.
+
+What pins what:
+  hand_cases        -- values worked out on paper (tests/golden/hand_cases.json)
+  onehot_matmul     -- one head selected: scores reduce to ReLU(K @ q), a
+                       numpy matmul; selection to numpy's stable argsort
+  positive_closed   -- all logits positive: ReLU is the identity, so the
+                       score is K @ (Q^T w), a numpy matmul
+  visible_closed    -- the count of returned keys with k >= T equals the
+                       closed form sum_t min(T, floor((t+1)/m))
+  causal            -- no returned key ends after its query
+  prefix            -- top-k is a prefix of top-(k+1)
+  brute_subsets     -- the returned set is the unique k-subset whose every
+                       member beats every non-member, found by enumeration
+  invariances       -- permuting heads (q and w together), scaling w by 2^j,
+                       w = 0 (all ties) -> indices 0..n-1
+  batch_independent -- sequence b's result does not depend on other sequences
+  fp8_matches_bf16  -- e4m3 inputs whose values are bf16-exact give the bf16 result
+"""
+from __future__ import annotations
+
+import itertools
+import json
+import os
+
+import numpy as np
+
+import oracle
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _bits(x) -> np.ndarray:
+    return synth.f32_to_bf16_bits(np.asarray(x, dtype=np.float32))
+
+
+def _f(bits) -> np.ndarray:
+    return synth.bf16_bits_to_f32(bits).astype(np.float64)
+
+
+def _int_problem(rng, B, S, T, H, D, lo=-3, hi=3):
+    q = _bits(rng.integers(lo, hi + 1, size=(B, S, H, D)))
+    kc = _bits(rng.integers(lo, hi + 1, size=(B, T, D)))
+    w = np.ldexp(1.0, -rng.integers(0, 7, size=(B, S, H))).astype(np.float32)
+    return q, kc, w
+
+
+def hand_cases(lib):
+    data = json.load(open(os.path.join(GOLDEN, "hand_cases.json")))
+    for case in data["cases"]:
+        B, S, T, H, D, m, k = (case[x] for x in ("B", "S", "T", "H", "D", "m", "k"))
+        q = np.zeros((B * S, H, D), dtype=np.float32)
+        w = np.zeros((B * S, H), dtype=np.float32)
+        for r, v in case["q"].items():
+            q[int(r)] = np.asarray(v, dtype=np.float32)
+        for r, v in case["w"].items():
+            w[int(r)] = np.asarray(v, dtype=np.float32)
+        kc = np.asarray(case["kc"], dtype=np.float32).reshape(B, T, D)
+        rows = np.array(sorted(int(r) for r in case["expect"]), dtype=np.int64)
+        idx, sc, _ = oracle.topk(_bits(q).reshape(B, S, H, D), _bits(kc), w.reshape(B, S, H), m, k,
+                                 rows=rows, lib=lib)
+        for i, r in enumerate(rows):
+            e = case["expect"][str(r)]
+            want_idx = np.asarray(e["idx"], dtype=np.int32)
+            want_sc = np.asarray([float(x) for x in e["score"]], dtype=np.float32)
+            assert np.array_equal(idx[i], want_idx), (case["name"], r, idx[i], want_idx)
+            assert np.array_equal(sc[i], want_sc), (case["name"], r, sc[i], want_sc)
+
+
+def onehot_matmul(lib, seed=11):
+    rng = np.random.default_rng(seed)
+    B, S, T, H, D, m, k = 1, 48, 12, 4, 8, 4, 5
+    q, kc, _ = _int_problem(rng, B, S, T, H, D)
+    for h0 in range(H):
+        w = np.zeros((B, S, H), dtype=np.float32)
+        w[..., h0] = 1.0
+        idx, sc, _ = oracle.topk(q, kc, w, m, k, lib=lib)
+        K = _f(kc[0])
+        for t in range(S):
+            n = min(T, (t + 1) // m)
+            s = np.maximum(K[:n] @ _f(q[0, t, h0]), 0.0)
+            order = np.argsort(-s, kind="stable")[:k]
+            want = np.full(k, -1, dtype=np.int32)
+            want[: len(order)] = order
+            assert np.array_equal(idx[t], want), (h0, t, idx[t], want)
+            assert np.array_equal(sc[t, : len(order)], s[order].astype(np.float32))
+
+
+def positive_closed(lib, seed=12):
+    rng = np.random.default_rng(seed)
+    B, S, T, H, D, m, k = 1, 40, 10, 3, 6, 4, 4
+    q, kc, w = _int_problem(rng, B, S, T, H, D, lo=1, hi=4)
+    idx, sc, sc64 = oracle.topk(q, kc, w, m, k, lib=lib)
+    K = _f(kc[0])
+    for t in range(S):
+        n = min(T, (t + 1) // m)
+        qw = _f(q[0, t]).T @ w[0, t].astype(np.float64)  # (D,)
+        s = K[:n] @ qw
+        order = np.argsort(-s, kind="stable")[:k]
+        assert np.array_equal(idx[t, : len(order)], order), (t, idx[t], order)
+        assert np.array_equal(sc64[t, : len(order)], s[order])
+
+
+def visible_closed(lib):
+    rng = np.random.default_rng(13)
+    for (S, T, m) in [(32, 8, 4), (30, 8, 4), (24, 5, 3), (17, 16, 1), (20, 4, 2)]:
+        H, D = 2, 4
+        q, kc, w = _int_problem(rng, 1, S, T, H, D)
+        idx, _, _ = oracle.topk(q, kc, w, m, T, lib=lib)
+        assert int((idx >= 0).sum()) == synth.visible_pairs(S, T, m), (S, T, m)
+        if S == m * T:
+            assert int((idx >= 0).sum()) == m * T * (T - 1) // 2 + T
+
+
+def causal(lib):
+    rng = np.random.default_rng(14)
+    S, T, m, k = 64, 16, 4, 6
+    q, kc, w = _int_problem(rng, 1, S, T, 2, 4)
+    idx, sc, _ = oracle.topk(q, kc, w, m, k, lib=lib)
+    for t in range(S):
+        valid = idx[t][idx[t] >= 0]
+        assert all(s * m + m - 1 <= t for s in valid), (t, valid)
+        n = min(T, (t + 1) // m)
+        assert len(valid) == min(k, n)
+        assert len(set(valid.tolist())) == len(valid)
+        assert np.all(np.isneginf(sc[t][idx[t] < 0]))
+
+
+def prefix(lib):
+    rng = np.random.default_rng(15)
+    S, T, m = 48, 12, 4
+    q, kc, w = _int_problem(rng, 1, S, T, 3, 5)
+    prev = None
+    for k in range(1, T + 2):
+        idx, _, _ = oracle.topk(q, kc, w, m, k, lib=lib)
+        if prev is not None:
+            assert np.array_equal(idx[:, : k - 1], prev), k
+        prev = idx
+
+
+def brute_subsets(lib):
+    rng = np.random.default_rng(16)
+    S, T, m = 36, 9, 4
+    q, kc, w = _int_problem(rng, 1, S, T, 2, 3, lo=-2, hi=2)
+    for t in (11, 23, 35):
+        n = min(T, (t + 1) // m)
+        sc = oracle.scores(q, kc, w, m, t, lib=lib)[:n]
+        key = [(sc[s], -s) for s in range(n)]
+        for k in range(1, n + 1):
+            idx, _, _ = oracle.topk(q, kc, w, m, k, rows=[t], lib=lib)
+            winners = [A for A in itertools.combinations(range(n), k)
+                       if min(key[a] for a in A) > max((key[b] for b in range(n) if b not in A),
+                                                       default=(-np.inf, -np.inf))]
+            assert len(winners) == 1
+            want = sorted(winners[0], key=lambda s: (-sc[s], s))
+            assert idx[0].tolist() == want, (t, k, idx[0], want)
+
+
+def invariances(lib):
+    rng = np.random.default_rng(17)
+    S, T, H, D, m, k = 40, 10, 4, 6, 4, 5
+    q, kc, w = _int_problem(rng, 1, S, T, H, D)
+    idx, sc, _ = oracle.topk(q, kc, w, m, k, lib=lib)
+    perm = rng.permutation(H)
+    idx2, sc2, _ = oracle.topk(np.ascontiguousarray(q[:, :, perm]), kc,
+                               np.ascontiguousarray(w[:, :, perm]), m, k, lib=lib)
+    assert np.array_equal(idx, idx2) and np.array_equal(sc, sc2)
+    for j in (-3, 2):
+        idx3, sc3, _ = oracle.topk(q, kc, (w * np.float32(2.0 ** j)).astype(np.float32), m, k, lib=lib)
+        assert np.array_equal(idx, idx3)
+        v = idx >= 0
+        assert np.array_equal(sc3[v], sc[v] * np.float32(2.0 ** j))
+    idx4, sc4, _ = oracle.topk(q, kc, np.zeros_like(w), m, k, lib=lib)
+    for t in range(S):
+        n = min(T, (t + 1) // m)
+        want = np.full(k, -1, dtype=np.int32)
+        want[: min(k, n)] = np.arange(min(k, n))
+        assert np.array_equal(idx4[t], want)
+        assert np.all(sc4[t, : min(k, n)] == 0.0)
+
+
+def batch_independent(lib):
+    rng = np.random.default_rng(18)
+    B, S, T, H, D, m, k = 3, 24, 6, 2, 4, 4, 4
+    q, kc, w = _int_problem(rng, B, S, T, H, D)
+    idx, sc, _ = oracle.topk(q, kc, w, m, k, lib=lib)
+    for b in range(B):
+        i1, s1, _ = oracle.topk(np.ascontiguousarray(q[b:b + 1]), np.ascontiguousarray(kc[b:b + 1]),
+                                np.ascontiguousarray(w[b:b + 1]), m, k, lib=lib)
+        assert np.array_equal(idx[b * S:(b + 1) * S], i1), b
+        assert np.array_equal(sc[b * S:(b + 1) * S], s1), b
+    # a different sequence's keys give a different answer somewhere
+    i_sw, _, _ = oracle.topk(q, np.ascontiguousarray(kc[::-1]), w, m, k, lib=lib)
+    assert not np.array_equal(i_sw, idx)
+
+
+def fp8_matches_bf16(lib):
+    rng = np.random.default_rng(19)
+    B, S, T, H, D, m, k = 1, 32, 8, 3, 16, 4, 5
+    q8 = rng.integers(0, 256, size=(B, S, H, D)).astype(np.uint8)
+    kc8 = rng.integers(0, 256, size=(B, T, D)).astype(np.uint8)
+    q8[(q8 & 0x7F) == 0x7F] = 0x10   # no NaN codes
+    kc8[(kc8 & 0x7F) == 0x7F] = 0x10
+    q_scale = np.ldexp(1.0, rng.integers(-2, 3, size=(B, S, H))).astype(np.float32)
+    kc_scale = np.ldexp(1.0, rng.integers(-2, 3, size=(B, T))).astype(np.float32)
+    w = rng.random((B, S, H)).astype(np.float32)
+    import torch
+    qv = torch.from_numpy(q8).view(torch.float8_e4m3fn).float().numpy() * q_scale[..., None]
+    kv = torch.from_numpy(kc8).view(torch.float8_e4m3fn).float().numpy() * kc_scale[..., None]
+    qb, kb = _bits(qv), _bits(kv)
+    assert np.array_equal(_f(qb), qv.astype(np.float64))  # e4m3 * 2^j is bf16-exact
+    i8, s8, _ = oracle.topk(q8, kc8, w, m, k, q_scale=q_scale, kc_scale=kc_scale, lib=lib)
+    ib, sb, _ = oracle.topk(qb, kb, w, m, k, lib=lib)
+    assert np.array_equal(i8, ib) and np.array_equal(s8, sb)
+
+
+ALL = [hand_cases, onehot_matmul, positive_closed, visible_closed, causal, prefix, brute_subsets,
+       invariances, batch_independent, fp8_matches_bf16]
