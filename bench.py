@@ -1,0 +1,340 @@
+#!/usr/bin/env python
+"""Benchmark of the streaming lightning-indexer top-k on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload v4flash]
+
+One step = one si_indexer_topk call over the whole workload (score every
+causally visible (query, key) pair with 64 indexer heads, keep the top-512
+per query).  Default workload: the V4-Flash shape, B=1, S=65,536, m=4
+(T=16,384), H_I=64, D=128, k=512, planted-boost Gaussian inputs, seed 3.
+Inputs are synthetic and resident in HBM before timing; q (1 GiB) exceeds the
+126 MB L2 and L2 is also flushed before every timed step.
+
+Under torchrun (N>1) each rank runs its own independent sequence of the same
+shape (weak scaling, no collective on the data path); the timing is the max
+over ranks.  `--impl reference` times the CPU oracle instead, on rank 0 only,
+on a bounded sample of query rows per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "visible q·k pairs/s (TFLOP/s, % bf16 TC peak) at S=65,536; peak HBM GB"
+FLOP_PER_PAIR = None  # 2 * H_I * D, set per workload
+
+
+def load_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("si_stream.cu", "si_ptx.cuh"):
+        h.update(open(os.path.join(ROOT, "streaming_top_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload: str):
+    """DRAM bytes per launch of the streaming kernel from the committed ncu
+    summary, if it was taken on the current kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", "stream_topk_traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    if d.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return d.get("per_launch_dram_bytes", {}).get(workload)
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+                power.append(float(f[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "samples": len(sm),
+                "power_w_max": max(power) if power else None, "reasons": sorted(reasons)}
+
+
+def config_dict(wl, n_gpus: int) -> dict:
+    return {"workload": f"{wl.name}: B={wl.B}, S={wl.S}, m={wl.m} (T={wl.T}), H_I={wl.H}, D={wl.D}, "
+                        f"k={wl.k}, {wl.kind} inputs, seed {wl.seed}",
+            "B_per_gpu": wl.B, "S": wl.S, "T": wl.T, "H_I": wl.H, "D": wl.D, "m": wl.m, "k": wl.k,
+            "visible_pairs_per_gpu": wl.visible_pairs(), "parallelism": f"independent sequences x{n_gpus}",
+            "l2": "q (1 GiB) > L2, and L2 flushed before each timed step"}
+
+
+# ------------------------------------------------------------------ CPU oracle
+def oracle_sample(wl, inp, rows) -> tuple[float, int]:
+    import oracle
+    t0 = time.perf_counter()
+    oracle.topk(inp["q"], inp["kc"], inp["w"], wl.m, wl.k, rows=rows)
+    dt = time.perf_counter() - t0
+    pairs = int(sum(min(wl.T, (int(r) % wl.S + 1) // wl.m) for r in rows))
+    return dt, pairs
+
+
+def run_reference(args, wl):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    inp = synth.make_inputs(wl)
+    per_step = args.ref_rows
+    allrows = synth.sample_rows(per_step * (args.steps + args.warmup), wl.m * 4, wl.S, seed=wl.seed + 77)
+    rng = np.random.default_rng(wl.seed)
+    rng.shuffle(allrows)
+    times, pairs = [], []
+    for i in range(args.warmup + args.steps):
+        rows = np.sort(allrows[i * per_step:(i + 1) * per_step])
+        dt, pr = oracle_sample(wl, inp, rows)
+        if i >= args.warmup:
+            times.append(dt)
+            pairs.append(pr)
+    tot_t, tot_p = sum(times), sum(pairs)
+    value = tot_p / tot_t
+    line = {
+        "metric": METRIC, "value": value, "unit": "pairs/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(wl, args.gpus), "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": "pairs/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{per_step} sampled query rows per step of the {wl.name} workload "
+                                   f"({tot_p // args.steps} visible pairs per step on average), "
+                                   "single-threaded C oracle, fp64, full sort"},
+        "e2e": {"value": value, "unit": "pairs/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+# ------------------------------------------------------------------ CUDA path
+def run_ours(args, wl):
+    import torch
+    import torch.distributed as dist
+
+    import streaming_top_b200 as si
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+
+    seed = wl.seed + 1000 * rank  # each rank: its own sequence of the same shape
+    inp = synth.make_inputs(wl, seed=seed)
+    q = torch.from_numpy(inp["q"].view(np.int16)).view(torch.bfloat16).to(dev)
+    kc = torch.from_numpy(inp["kc"].view(np.int16)).view(torch.bfloat16).to(dev)
+    w = torch.from_numpy(inp["w"]).to(dev)
+    out_idx = torch.empty((wl.B, wl.S, wl.k), dtype=torch.int32, device=dev)
+    out_score = torch.empty((wl.B, wl.S, wl.k), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)  # > 126 MB L2
+    stream = torch.cuda.current_stream(dev)
+    torch.cuda.synchronize(dev)
+    torch.cuda.reset_peak_memory_stats(dev)
+
+    def step():
+        si.indexer_topk(q, kc, w, wl.m, wl.k, out_idx=out_idx, out_score=out_score, stream=stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    if si.device_status(stream) != si.SI_OK:
+        raise RuntimeError("device error during warm-up")
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    sampler = ClockSampler(local if "CUDA_VISIBLE_DEVICES" not in os.environ else
+                           int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local]))
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    time.sleep(0.3)
+    wall0 = time.perf_counter()
+    for e0, e1 in evs:
+        flush.zero_()
+        e0.record(stream)
+        step()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    wall = time.perf_counter() - wall0
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    st = si.device_status(stream)
+    if st != si.SI_OK:
+        raise RuntimeError(f"device error during the timed steps: {st}")
+    ms = [e0.elapsed_time(e1) for e0, e1 in evs]
+    ms_step = sum(ms) / len(ms)
+    peak_mem = torch.cuda.max_memory_allocated(dev)
+    if world > 1:
+        t = torch.tensor([ms_step], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step = float(t.item())
+
+    # end to end through the host-buffer API: H2D inputs, kernel, D2H results
+    hq = torch.from_numpy(inp["q"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    hk = torch.from_numpy(inp["kc"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    hw = torch.from_numpy(inp["w"]).pin_memory()
+    bufs = {}
+    for _ in range(max(1, args.warmup)):
+        si.indexer_topk_host(hq, hk, hw, wl.m, wl.k, device=dev, bufs=bufs)
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    for e0, e1 in e2e_ev:
+        e0.record(stream)
+        si.indexer_topk_host(hq, hk, hw, wl.m, wl.k, device=dev, bufs=bufs, sync=False)
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev) / args.steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = hq.numel() * 2 + hk.numel() * 2 + hw.numel() * 4
+    d2h = out_idx.numel() * 4 + out_score.numel() * 4
+    del bufs
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    P = wl.visible_pairs()
+    flop_pair = 2 * wl.H * wl.D
+    peaks = load_peaks()
+    value = world * P / (ms_step * 1e-3)
+    tflops = P * flop_pair / (ms_step * 1e-3) / 1e12
+    alg_bytes = q.numel() * 2 + kc.numel() * 2 + w.numel() * 4 + out_idx.numel() * 4 + out_score.numel() * 4
+    traffic = ncu_traffic(wl.name)
+    cpu = None
+    if world == 1:
+        rows = synth.sample_rows(4096, wl.m * 4, wl.S, seed=wl.seed + 99)
+        rng = np.random.default_rng(wl.seed)
+        rng.shuffle(rows)
+        done, t_tot, p_tot = 0, 0.0, 0
+        while t_tot < args.cpu_seconds and done < len(rows):
+            chunk = np.sort(rows[done:done + 16])
+            dt, pr = oracle_sample(wl, inp, chunk)
+            t_tot += dt
+            p_tot += pr
+            done += len(chunk)
+        cpu = {"value": p_tot / t_tot, "unit": "pairs/s", "cores": 1, "kind": "oracle",
+               "sample": f"{done} uniformly sampled query rows of the {wl.name} workload ({p_tot} visible "
+                         f"pairs, {t_tot:.1f} s), single-threaded C oracle, fp64, full sort"}
+    line = {
+        "metric": METRIC, "value": value, "unit": "pairs/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(wl, world),
+        "tflops": tflops,
+        "frac_bf16_peak": tflops / peaks["bf16_tflops"],
+        "frac_bf16_peak_sustained": tflops / peaks["bf16_tflops_sustained"] if peaks["bf16_tflops_sustained"] else None,
+        "hbm_gbs": alg_bytes / (ms_step * 1e-3) / 1e9,
+        "frac_hbm": alg_bytes / (ms_step * 1e-3) / 1e9 / peaks["hbm_gbs"],
+        "peak_hbm_gb": peak_mem / 1e9,
+        "hbm_breakdown_gb": {"q": q.numel() * 2 / 1e9, "kc": kc.numel() * 2 / 1e9, "w": w.numel() * 4 / 1e9,
+                             "out_idx": out_idx.numel() * 4 / 1e9, "out_score": out_score.numel() * 4 / 1e9,
+                             "l2_flush_buffer": flush.numel() / 1e9, "library_workspace": 0.0},
+        "roofline": {"bound": "tensor", "kernel": "stream_topk_kernel", "achieved": tflops,
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": tflops / peaks["bf16_tflops"],
+                     "peak_source": f"{peaks['source']} bf16 dense matmul, burst",
+                     "traffic": traffic, "algorithmic_bytes": alg_bytes},
+        "cpu_baseline": cpu,
+        "e2e": {"value": world * P / (e2e_ms * 1e-3), "unit": "pairs/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+        "wall_s_timed": wall,
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def main() -> int:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="v4flash", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-rows", type=int, default=32)
+    args = ap.parse_args()
+    wl = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, wl)
+    return run_ours(args, wl)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

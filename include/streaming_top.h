@@ -1,0 +1,123 @@
+/*
+ * streaming_top -- C ABI of the B200 (sm_100a) CSA lightning-indexer top-k.
+ *
+ * The operation (StreamIndex, "Memory-Bounded Compressed Sparse Attention via
+ * Streaming Top-k", abstract: the lightning indexer scores the compressed keys
+ * and the top-k are selected per query, by a chunked partition-merge top-k that
+ * never materialises the [B, S, H_I, T] fp32 score tensor).  The scoring
+ * function is the DeepSeek-V3.2 lightning-indexer form (the lineage the
+ * DeepSeek-V4.1 sparse-attention page gives the indexer, section "indexer"):
+ *
+ *     I[b,t,s] = sum_{h < H_I} w[b,t,h] * ReLU( sum_{d < D} q[b,t,h,d] * kc[b,s,d] )
+ *
+ * Compressed key s covers tokens [s*m, s*m+m-1] and is visible to query t iff
+ * s*m+m-1 <= t and s < T.  For every (b, t) the result is the visible keys
+ * with the k largest scores, sorted by score descending with the lower index
+ * winning ties; when fewer than k keys are visible the tail is index -1 and
+ * score -inf.
+ *
+ * Conventions shared by every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller, dense
+ *     row-major (C order), 16-byte aligned.  The library never frees or keeps
+ *     them after the call returns.
+ *   - Calls are asynchronous: they validate arguments on the host, enqueue
+ *     work on `stream` (a cudaStream_t; NULL means the legacy default stream)
+ *     and return.  A validation failure returns a status synchronously and
+ *     enqueues nothing.  Device-side failures (a bounded wait that ran out) are
+ *     reported by si_device_status().
+ *   - The message of the last failure on the calling host thread is available
+ *     from si_last_error().
+ */
+#ifndef STREAMING_TOP_H
+#define STREAMING_TOP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SI_API __attribute__((visibility("default")))
+#else
+#define SI_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum si_status {
+  SI_OK = 0,
+  SI_ERR_INVALID_ARGUMENT = 1, /* null pointer, non-positive size, misaligned pointer */
+  SI_ERR_UNSUPPORTED = 2,      /* valid but outside what the kernels implement (D, H_I, k, key tile) */
+  SI_ERR_OUT_OF_MEMORY = 3,    /* the path's memory need exceeds free device memory */
+  SI_ERR_CUDA = 4,             /* a CUDA runtime/driver call failed; see si_last_error() */
+  SI_ERR_TIMEOUT = 5           /* a kernel's bounded wait ran out; the kernel exited early */
+} si_status;
+
+typedef enum si_dtype {
+  SI_DTYPE_BF16 = 0,     /* q, kc are bf16 */
+  SI_DTYPE_FP8_E4M3 = 1  /* q, kc are OCP fp8 e4m3 codes with per-row fp32 scales */
+} si_dtype;
+
+/* Options of si_indexer_topk_ex.  Zero-initialise, then set what you need. */
+typedef struct si_options {
+  si_dtype dtype;        /* SI_DTYPE_BF16 (default) or SI_DTYPE_FP8_E4M3 */
+  const float* q_scale;  /* fp8 only: [B,S,H_I] fp32 > 0, value = code * scale (device) */
+  const float* kc_scale; /* fp8 only: [B,T] fp32 > 0 (device) */
+  int query_chunk;       /* queries per launch of the chunk driver; 0 = all S in one launch.
+                            Must be a multiple of 4 otherwise. */
+  int key_tile;          /* keys per partition of the partition-merge: 64 or a multiple
+                            of 128 up to 1024; 0 = 256 */
+  void* workspace;       /* optional caller-owned device scratch, >= si_indexer_workspace_size() */
+  size_t workspace_bytes;
+} si_options;
+
+/*
+ * Streaming indexer top-k (the hot path).  Never allocates the
+ * [B,S,H_I,T] score tensor.
+ *   q       [B, S, H_I, D] bf16     kc [B, T, D] bf16     w [B, S, H_I] fp32
+ *   out_idx [B, S, k] int32 (device, written)
+ *   out_score [B, S, k] fp32 (device, written; may be NULL)
+ * Supported: D == 128, H_I == 64, 1 <= k <= 2048, m >= 1, B, S, T >= 1.
+ * Other shapes return SI_ERR_UNSUPPORTED.
+ */
+SI_API si_status si_indexer_topk(const void* q, const void* kc, const float* w, int B, int S, int T,
+                          int H_I, int D, int m, int k, int32_t* out_idx, float* out_score,
+                          void* stream);
+
+/* As si_indexer_topk, with options (dtype, fp8 scales, query chunk, key tile,
+ * workspace).  opt may be NULL (defaults). */
+SI_API si_status si_indexer_topk_ex(const void* q, const void* kc, const float* w, int B, int S, int T,
+                             int H_I, int D, int m, int k, int32_t* out_idx, float* out_score,
+                             void* stream, const si_options* opt);
+
+/*
+ * Materialize path (in-library ground truth for small S, the method the
+ * pages contrast with): writes the full [B,S,H_I,T] fp32 logits, reduces them
+ * to [B,S,T] scores, then fully sorts every row.  Same arguments and results
+ * as si_indexer_topk; any D >= 1 and H_I >= 1; T <= 16384.  Needs
+ * 4*B*S*T*(H_I+1) bytes of scratch (taken from opt->workspace when given,
+ * else allocated on `stream`); returns SI_ERR_OUT_OF_MEMORY without
+ * allocating when that exceeds the free device memory.
+ */
+SI_API si_status si_indexer_materialize(const void* q, const void* kc, const float* w, int B, int S,
+                                 int T, int H_I, int D, int m, int k, int32_t* out_idx,
+                                 float* out_score, void* stream, const si_options* opt);
+
+/* Scratch bytes a call with these arguments needs (0 if none).  materialize
+ * selects the materialize path's need. */
+SI_API size_t si_indexer_workspace_size(int B, int S, int T, int H_I, int D, int m, int k, int materialize,
+                                 const si_options* opt);
+
+/* Waits for `stream`, then returns SI_ERR_TIMEOUT (and clears the record) if
+ * any kernel of this library timed out in a bounded wait since the last call,
+ * else the stream's own error state (SI_OK or SI_ERR_CUDA). */
+SI_API si_status si_device_status(void* stream);
+
+SI_API const char* si_status_string(si_status s);
+SI_API const char* si_last_error(void); /* thread-local; "" when none */
+SI_API int si_version(void);            /* major*10000 + minor*100 + patch */
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* STREAMING_TOP_H */

@@ -1,0 +1,213 @@
+"""Python binding of the B200 CSA lightning-indexer top-k library.
+
+Argument marshalling only: every step of the indexer runs in the CUDA kernels
+of ``libstreaming_top.so`` (built by ``python streaming_top_b200/build.py``).
+Tensors are torch CUDA tensors; torch provides device memory and streams.
+There is no CPU fallback: without the built library this module fails to
+import.
+
+    q   [B, S, H_I, D] bf16 (or uint8 e4m3 codes + q_scale [B, S, H_I] fp32)
+    kc  [B, T, D]      bf16 (or uint8 e4m3 codes + kc_scale [B, T] fp32)
+    w   [B, S, H_I]    fp32
+    ->  idx [B, S, k] int32 (-1 padded), score [B, S, k] fp32 (-inf padded)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libstreaming_top.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python streaming_top_b200/build.py` "
+                      "(the indexer has no CPU fallback)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+SI_OK, SI_ERR_INVALID_ARGUMENT, SI_ERR_UNSUPPORTED, SI_ERR_OUT_OF_MEMORY, SI_ERR_CUDA, SI_ERR_TIMEOUT = range(6)
+SI_DTYPE_BF16, SI_DTYPE_FP8_E4M3 = 0, 1
+
+_vp, _i, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+
+
+class Options(ctypes.Structure):
+    _fields_ = [("dtype", _i), ("q_scale", _vp), ("kc_scale", _vp), ("query_chunk", _i),
+                ("key_tile", _i), ("workspace", _vp), ("workspace_bytes", _sz)]
+
+
+_ARGS = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp]
+_lib.si_indexer_topk.restype = _i
+_lib.si_indexer_topk.argtypes = _ARGS
+_lib.si_indexer_topk_ex.restype = _i
+_lib.si_indexer_topk_ex.argtypes = _ARGS + [ctypes.POINTER(Options)]
+_lib.si_indexer_materialize.restype = _i
+_lib.si_indexer_materialize.argtypes = _ARGS + [ctypes.POINTER(Options)]
+_lib.si_indexer_workspace_size.restype = _sz
+_lib.si_indexer_workspace_size.argtypes = [_i] * 8 + [ctypes.POINTER(Options)]
+_lib.si_device_status.restype = _i
+_lib.si_device_status.argtypes = [_vp]
+_lib.si_status_string.restype = ctypes.c_char_p
+_lib.si_status_string.argtypes = [_i]
+_lib.si_last_error.restype = ctypes.c_char_p
+_lib.si_last_error.argtypes = []
+_lib.si_version.restype = _i
+_lib.si_test_stream_timeout.restype = _i
+_lib.si_test_stream_timeout.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, ctypes.c_ulonglong]
+
+
+class SIError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = _lib.si_last_error().decode(errors="replace")
+        super().__init__(f"{where}: {_lib.si_status_string(status).decode()}: {msg}")
+
+
+def _check(st: int, where: str) -> None:
+    if st != SI_OK:
+        raise SIError(st, where)
+
+
+def lib():
+    """The ctypes handle on libstreaming_top.so."""
+    return _lib
+
+
+def version() -> int:
+    return _lib.si_version()
+
+
+def _stream_ptr(stream) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _shapes(q, kc, w):
+    if q.dim() != 4 or kc.dim() != 3 or w.dim() != 3:
+        raise ValueError("q [B,S,H,D], kc [B,T,D], w [B,S,H] expected")
+    B, S, H, D = q.shape
+    if kc.shape[0] != B or kc.shape[2] != D or tuple(w.shape) != (B, S, H):
+        raise ValueError(f"shape mismatch q{tuple(q.shape)} kc{tuple(kc.shape)} w{tuple(w.shape)}")
+    for name, t in (("q", q), ("kc", kc), ("w", w)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if w.dtype != torch.float32:
+        raise ValueError("w must be float32")
+    return B, S, kc.shape[1], H, D
+
+
+def _outputs(B, S, k, device, out_idx, out_score, with_score):
+    if out_idx is None:
+        out_idx = torch.empty((B, S, k), dtype=torch.int32, device=device)
+    if out_score is None and with_score:
+        out_score = torch.empty((B, S, k), dtype=torch.float32, device=device)
+    return out_idx, out_score
+
+
+def _options(q, q_scale, kc_scale, query_chunk, key_tile, workspace=None):
+    o = Options()
+    if q.dtype == torch.bfloat16:
+        o.dtype = SI_DTYPE_BF16
+    elif q.dtype in (torch.uint8, torch.float8_e4m3fn):
+        if q_scale is None or kc_scale is None:
+            raise ValueError("fp8 inputs need q_scale and kc_scale")
+        o.dtype = SI_DTYPE_FP8_E4M3
+        o.q_scale = q_scale.data_ptr()
+        o.kc_scale = kc_scale.data_ptr()
+    else:
+        raise ValueError(f"unsupported q dtype {q.dtype}")
+    o.query_chunk = int(query_chunk)
+    o.key_tile = int(key_tile)
+    if workspace is not None:
+        o.workspace = workspace.data_ptr()
+        o.workspace_bytes = workspace.numel() * workspace.element_size()
+    return o
+
+
+def indexer_topk(q, kc, w, m: int, k: int, *, q_scale=None, kc_scale=None, query_chunk: int = 0,
+                 key_tile: int = 0, out_idx=None, out_score=None, with_score: bool = True,
+                 stream=None):
+    """Streaming indexer top-k (``si_indexer_topk_ex``).  Returns (idx, score)."""
+    B, S, T, H, D = _shapes(q, kc, w)
+    out_idx, out_score = _outputs(B, S, k, q.device, out_idx, out_score, with_score)
+    o = _options(q, q_scale, kc_scale, query_chunk, key_tile)
+    st = _lib.si_indexer_topk_ex(q.data_ptr(), kc.data_ptr(), w.data_ptr(), B, S, T, H, D, m, k,
+                                 out_idx.data_ptr(), out_score.data_ptr() if out_score is not None else None,
+                                 _stream_ptr(stream), ctypes.byref(o))
+    _check(st, "si_indexer_topk_ex")
+    return out_idx, out_score
+
+
+def indexer_materialize(q, kc, w, m: int, k: int, *, out_idx=None, out_score=None,
+                        with_score: bool = True, workspace=None, stream=None):
+    """Materialize-path ground truth (``si_indexer_materialize``)."""
+    B, S, T, H, D = _shapes(q, kc, w)
+    out_idx, out_score = _outputs(B, S, k, q.device, out_idx, out_score, with_score)
+    o = _options(q, None, None, 0, 0, workspace)
+    st = _lib.si_indexer_materialize(q.data_ptr(), kc.data_ptr(), w.data_ptr(), B, S, T, H, D, m, k,
+                                     out_idx.data_ptr(),
+                                     out_score.data_ptr() if out_score is not None else None,
+                                     _stream_ptr(stream), ctypes.byref(o))
+    _check(st, "si_indexer_materialize")
+    return out_idx, out_score
+
+
+def workspace_size(B, S, T, H, D, m, k, materialize: bool = False) -> int:
+    return int(_lib.si_indexer_workspace_size(B, S, T, H, D, m, k, int(materialize), None))
+
+
+def device_status(stream=None) -> int:
+    """Synchronise the stream; return SI_OK or the status of a device-side failure."""
+    return int(_lib.si_device_status(_stream_ptr(stream)))
+
+
+def indexer_topk_host(q, kc, w, m: int, k: int, *, q_scale=None, kc_scale=None, device="cuda",
+                      query_chunk: int = 0, key_tile: int = 0, bufs: dict | None = None,
+                      sync: bool = True):
+    """End-to-end call on HOST tensors (pinned for best speed): copies the
+    inputs to the device, runs the streaming top-k, copies (idx, score) back.
+    `bufs` may hold reusable device buffers from a previous call.  With
+    sync=False the copies back are only enqueued on the current stream."""
+    bufs = {} if bufs is None else bufs
+    stream = torch.cuda.current_stream(device)
+
+    def dev(name, t):
+        d = bufs.get(name)
+        if d is None or d.shape != t.shape or d.dtype != t.dtype:
+            d = torch.empty(t.shape, dtype=t.dtype, device=device)
+            bufs[name] = d
+        d.copy_(t, non_blocking=True)
+        return d
+
+    qd, kd, wd = dev("q", q), dev("kc", kc), dev("w", w)
+    qs = dev("q_scale", q_scale) if q_scale is not None else None
+    ks = dev("kc_scale", kc_scale) if kc_scale is not None else None
+    B, S = q.shape[0], q.shape[1]
+    oi = bufs.get("out_idx")
+    os_ = bufs.get("out_score")
+    if oi is None or oi.shape != (B, S, k):
+        oi = bufs["out_idx"] = torch.empty((B, S, k), dtype=torch.int32, device=device)
+        os_ = bufs["out_score"] = torch.empty((B, S, k), dtype=torch.float32, device=device)
+    indexer_topk(qd, kd, wd, m, k, q_scale=qs, kc_scale=ks, query_chunk=query_chunk,
+                 key_tile=key_tile, out_idx=oi, out_score=os_, stream=stream)
+    hi = bufs.get("h_idx")
+    hs = bufs.get("h_score")
+    if hi is None or hi.shape != oi.shape:
+        hi = bufs["h_idx"] = torch.empty(oi.shape, dtype=oi.dtype, pin_memory=True)
+        hs = bufs["h_score"] = torch.empty(os_.shape, dtype=os_.dtype, pin_memory=True)
+    hi.copy_(oi, non_blocking=True)
+    hs.copy_(os_, non_blocking=True)
+    if sync:
+        stream.synchronize()
+    return hi, hs
+
+
+def test_stream_timeout(q, kc, w, m: int, k: int, out_idx, wait_limit_ns: int, stream=None) -> int:
+    """Test hook: run the streaming kernel with one key tile withheld and a
+    short bounded-wait limit; returns the launch status (the timeout itself is
+    reported by device_status())."""
+    B, S, T, H, D = _shapes(q, kc, w)
+    return int(_lib.si_test_stream_timeout(q.data_ptr(), kc.data_ptr(), w.data_ptr(), B, S, T, m, k,
+                                           out_idx.data_ptr(), _stream_ptr(stream), wait_limit_ns))

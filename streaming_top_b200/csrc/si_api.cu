@@ -1,0 +1,227 @@
+// C-ABI entry points of the indexer top-k library: argument validation,
+// error reporting, the device error record and TMA tensor-map encoding.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "si_internal.h"
+
+namespace si {
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+// Error record written by the kernels of this library (per device).
+__device__ int g_device_error[4];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+int* g_err_ptr[kMaxDevices] = {};
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+std::once_flag g_encode_once;
+cudaError_t g_encode_err = cudaSuccess;
+
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;  // 2 s per bounded wait
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+}  // namespace
+
+si_status fail(si_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+si_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(SI_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+si_status device_error_record(int** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(SI_ERR_UNSUPPORTED, "device index %d", dev);
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_err_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_device_error);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(error record)");
+    g_err_ptr[dev] = static_cast<int*>(p);
+  }
+  *out = g_err_ptr[dev];
+  return SI_OK;
+}
+
+si_status encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
+                         uint64_t inner, uint64_t outer, uint64_t row_bytes, uint32_t box_inner,
+                         uint32_t box_outer) {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    g_encode_err = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+    if (g_encode_err == cudaSuccess && q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  });
+  if (!g_encode) return fail(SI_ERR_CUDA, "cuTensorMapEncodeTiled unavailable (%s)", cudaGetErrorString(g_encode_err));
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = g_encode(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SI_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", static_cast<int>(r));
+  return SI_OK;
+}
+
+namespace {
+
+si_status check_common(const void* q, const void* kc, const float* w, int B, int S, int T, int H,
+                       int D, int m, int k, const int32_t* out_idx, const float* out_score) {
+  if (!q || !kc || !w || !out_idx)
+    return fail(SI_ERR_INVALID_ARGUMENT, "q, kc, w and out_idx must be non-null device pointers");
+  if (B < 1 || S < 1 || T < 1 || H < 1 || D < 1 || m < 1 || k < 1)
+    return fail(SI_ERR_INVALID_ARGUMENT, "B, S, T, H_I, D, m, k must be >= 1 (got %d %d %d %d %d %d %d)",
+                B, S, T, H, D, m, k);
+  if (!aligned(q, 16) || !aligned(kc, 16) || !aligned(w, 16) || !aligned(out_idx, 4) ||
+      (out_score && !aligned(out_score, 4)))
+    return fail(SI_ERR_INVALID_ARGUMENT, "q, kc, w must be 16-byte aligned; outputs 4-byte aligned");
+  return SI_OK;
+}
+
+}  // namespace
+}  // namespace si
+
+using namespace si;
+
+extern "C" {
+
+si_status si_indexer_topk_ex(const void* q, const void* kc, const float* w, int B, int S, int T,
+                             int H_I, int D, int m, int k, int32_t* out_idx, float* out_score,
+                             void* stream, const si_options* opt) {
+  si_status st = check_common(q, kc, w, B, S, T, H_I, D, m, k, out_idx, out_score);
+  if (st != SI_OK) return st;
+  si_options o;
+  std::memset(&o, 0, sizeof o);
+  if (opt) o = *opt;
+  if (o.dtype != SI_DTYPE_BF16 && o.dtype != SI_DTYPE_FP8_E4M3)
+    return fail(SI_ERR_INVALID_ARGUMENT, "unknown dtype %d", static_cast<int>(o.dtype));
+  if (o.dtype == SI_DTYPE_FP8_E4M3 && (!o.q_scale || !o.kc_scale))
+    return fail(SI_ERR_INVALID_ARGUMENT, "fp8 inputs need q_scale and kc_scale");
+  const int key_tile = o.key_tile ? o.key_tile : 256;
+  if (!(key_tile == 64 || (key_tile % 128 == 0 && key_tile >= 128 && key_tile <= 1024)))
+    return fail(SI_ERR_INVALID_ARGUMENT, "key_tile must be 64 or a multiple of 128 up to 1024 (got %d)", key_tile);
+  if (o.query_chunk < 0 || (o.query_chunk % 4) != 0)
+    return fail(SI_ERR_INVALID_ARGUMENT, "query_chunk must be 0 or a positive multiple of 4 (got %d)", o.query_chunk);
+  if (D != 128 || H_I != 64)
+    return fail(SI_ERR_UNSUPPORTED, "streaming path implements D=128, H_I=64 (got D=%d, H_I=%d)", D, H_I);
+  if (k > 2048) return fail(SI_ERR_UNSUPPORTED, "k <= 2048 (got %d)", k);
+  if (static_cast<long long>(B) * S * H_I > 0x7FFFFFFFll || static_cast<long long>(B) * T > 0x7FFFFFFFll)
+    return fail(SI_ERR_UNSUPPORTED, "B*S*H_I and B*T must fit in 31 bits");
+  StreamConfig cfg;
+  cfg.query_chunk = o.query_chunk;
+  cfg.key_tile = key_tile;
+  cfg.fp8 = o.dtype == SI_DTYPE_FP8_E4M3;
+  cfg.q_scale = o.q_scale;
+  cfg.kc_scale = o.kc_scale;
+  cfg.wait_limit_ns = kDefaultWaitLimitNs;
+  cfg.test_withhold = 0;
+  return launch_stream_topk(q, kc, w, B, S, T, H_I, D, m, k, out_idx, out_score,
+                            static_cast<cudaStream_t>(stream), cfg);
+}
+
+si_status si_indexer_topk(const void* q, const void* kc, const float* w, int B, int S, int T,
+                          int H_I, int D, int m, int k, int32_t* out_idx, float* out_score,
+                          void* stream) {
+  return si_indexer_topk_ex(q, kc, w, B, S, T, H_I, D, m, k, out_idx, out_score, stream, nullptr);
+}
+
+// Test entry point (not declared in the public header): runs the streaming
+// kernel with a short wait limit and one key tile withheld, so that its
+// bounded waits run out and it exits with SI_ERR_TIMEOUT recorded.
+si_status si_test_stream_timeout(const void* q, const void* kc, const float* w, int B, int S, int T,
+                                 int m, int k, int32_t* out_idx, void* stream,
+                                 unsigned long long wait_limit_ns) {
+  si_status st = check_common(q, kc, w, B, S, T, 64, 128, m, k, out_idx, nullptr);
+  if (st != SI_OK) return st;
+  StreamConfig cfg;
+  cfg.query_chunk = 0;
+  cfg.key_tile = 256;
+  cfg.fp8 = 0;
+  cfg.q_scale = nullptr;
+  cfg.kc_scale = nullptr;
+  cfg.wait_limit_ns = wait_limit_ns;
+  cfg.test_withhold = 1;
+  return launch_stream_topk(q, kc, w, B, S, T, 64, 128, m, k, out_idx, nullptr,
+                            static_cast<cudaStream_t>(stream), cfg);
+}
+
+si_status si_indexer_materialize(const void* q, const void* kc, const float* w, int B, int S,
+                                 int T, int H_I, int D, int m, int k, int32_t* out_idx,
+                                 float* out_score, void* stream, const si_options* opt) {
+  si_status st = check_common(q, kc, w, B, S, T, H_I, D, m, k, out_idx, out_score);
+  if (st != SI_OK) return st;
+  if (opt && opt->dtype != SI_DTYPE_BF16)
+    return fail(SI_ERR_UNSUPPORTED, "materialize path takes bf16 inputs");
+  if (T > 16384) return fail(SI_ERR_UNSUPPORTED, "materialize path sorts rows of T <= 16384 (got %d)", T);
+  return launch_materialize(q, kc, w, B, S, T, H_I, D, m, k, out_idx, out_score,
+                            static_cast<cudaStream_t>(stream), opt ? opt->workspace : nullptr,
+                            opt ? opt->workspace_bytes : 0);
+}
+
+size_t si_indexer_workspace_size(int B, int S, int T, int H_I, int D, int m, int k, int materialize,
+                                 const si_options* opt) {
+  (void)D;
+  (void)m;
+  (void)k;
+  (void)opt;
+  if (B < 1 || S < 1 || T < 1 || H_I < 1) return 0;
+  return materialize ? materialize_workspace_bytes(B, S, T, H_I) : 0;
+}
+
+si_status si_device_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int* rec = nullptr;
+  si_status st = device_error_record(&rec);
+  if (st != SI_OK) return st;
+  int h[4] = {0, 0, 0, 0};
+  e = cudaMemcpy(h, rec, sizeof h, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device error record");
+  if (h[0] != 0) {
+    e = cudaMemset(rec, 0, sizeof h);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the device error record");
+    return fail(static_cast<si_status>(h[0]), "a kernel's bounded wait ran out (site %d)", h[1]);
+  }
+  return SI_OK;
+}
+
+const char* si_status_string(si_status s) {
+  switch (s) {
+    case SI_OK: return "SI_OK";
+    case SI_ERR_INVALID_ARGUMENT: return "SI_ERR_INVALID_ARGUMENT";
+    case SI_ERR_UNSUPPORTED: return "SI_ERR_UNSUPPORTED";
+    case SI_ERR_OUT_OF_MEMORY: return "SI_ERR_OUT_OF_MEMORY";
+    case SI_ERR_CUDA: return "SI_ERR_CUDA";
+    case SI_ERR_TIMEOUT: return "SI_ERR_TIMEOUT";
+  }
+  return "SI_ERR_UNKNOWN";
+}
+
+const char* si_last_error(void) { return g_last_error; }
+
+int si_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,87 @@
+"""The C-ABI library loads and exports every function the headers declare;
+argument validation happens on the host (no GPU needed for these calls)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+import streaming_top_b200 as si
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = []
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names += re.findall(r"SI_API\s+[\w\s\*]+?\b(si_\w+)\s*\(", src)
+    return sorted(set(names))
+
+
+def test_headers_declare_the_entry_points():
+    names = declared_functions()
+    for n in ("si_indexer_topk", "si_indexer_topk_ex", "si_indexer_materialize",
+              "si_indexer_workspace_size", "si_device_status", "si_status_string", "si_last_error",
+              "si_version"):
+        assert n in names
+
+
+@pytest.mark.parametrize("name", declared_functions())
+def test_library_exports(name):
+    assert hasattr(si.lib(), name), name
+
+
+def test_status_strings_and_version():
+    L = si.lib()
+    assert L.si_status_string(si.SI_ERR_TIMEOUT) == b"SI_ERR_TIMEOUT"
+    assert L.si_status_string(0) == b"SI_OK"
+    assert si.version() >= 100
+
+
+# Fake, 16-byte aligned addresses: every call below is rejected by host-side
+# validation before any CUDA call, so nothing ever dereferences them.
+P = 4096
+
+
+def _call(q=P, kc=P, w=P, B=1, S=64, T=16, H=64, D=128, m=4, k=8, out=P, opt=None):
+    o = ctypes.byref(opt) if opt is not None else None
+    return si.lib().si_indexer_topk_ex(q, kc, w, B, S, T, H, D, m, k, out, None, None, o)
+
+
+@pytest.mark.parametrize("kw,status", [
+    ({"q": None}, si.SI_ERR_INVALID_ARGUMENT),
+    ({"out": None}, si.SI_ERR_INVALID_ARGUMENT),
+    ({"S": 0}, si.SI_ERR_INVALID_ARGUMENT),
+    ({"k": 0}, si.SI_ERR_INVALID_ARGUMENT),
+    ({"m": 0}, si.SI_ERR_INVALID_ARGUMENT),
+    ({"q": P + 8}, si.SI_ERR_INVALID_ARGUMENT),
+    ({"D": 64}, si.SI_ERR_UNSUPPORTED),
+    ({"H": 32}, si.SI_ERR_UNSUPPORTED),
+    ({"k": 4096}, si.SI_ERR_UNSUPPORTED),
+])
+def test_validation(kw, status):
+    assert _call(**kw) == status
+    assert si.lib().si_last_error()  # a message was recorded
+
+
+@pytest.mark.parametrize("field,value", [("key_tile", 100), ("key_tile", 2048), ("query_chunk", 6),
+                                         ("query_chunk", -4), ("dtype", 7)])
+def test_option_validation(field, value):
+    o = si.Options()
+    setattr(o, field, value)
+    assert _call(opt=o) == si.SI_ERR_INVALID_ARGUMENT
+
+
+def test_fp8_needs_scales():
+    o = si.Options()
+    o.dtype = si.SI_DTYPE_FP8_E4M3
+    assert _call(opt=o) == si.SI_ERR_INVALID_ARGUMENT
+
+
+def test_workspace_size():
+    assert si.workspace_size(1, 1024, 256, 64, 128, 4, 64, materialize=False) == 0
+    need = si.workspace_size(1, 1024, 256, 64, 128, 4, 64, materialize=True)
+    assert need >= 4 * 1024 * 256 * 65

@@ -1,0 +1,218 @@
+"""Parity of the CUDA streaming top-k (and the in-library materialize path)
+with the CPU oracle, through the C ABI, on a B200."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+import streaming_top_b200 as si  # noqa: E402  (fails loudly when the library is missing)
+
+
+def _dev(inp):
+    q = torch.from_numpy(inp["q"].view(np.int16)).view(torch.bfloat16).cuda()
+    kc = torch.from_numpy(inp["kc"].view(np.int16)).view(torch.bfloat16).cuda()
+    w = torch.from_numpy(inp["w"]).cuda()
+    return q, kc, w
+
+
+def _run(inp, m, k, **kw):
+    q, kc, w = _dev(inp)
+    idx, sc = si.indexer_topk(q, kc, w, m, k, **kw)
+    assert si.device_status() == si.SI_OK
+    return idx.cpu().numpy().reshape(-1, k), sc.cpu().numpy().reshape(-1, k)
+
+
+def _mat(inp, m, k):
+    q, kc, w = _dev(inp)
+    idx, sc = si.indexer_materialize(q, kc, w, m, k)
+    assert si.device_status() == si.SI_OK
+    return idx.cpu().numpy().reshape(-1, k), sc.cpu().numpy().reshape(-1, k)
+
+
+def _int_inputs(B, S, T, seed, H=64, D=128):
+    q = synth.matrix(B * S * H, D, seed, synth.TENSOR_Q, "int").reshape(B, S, H, D)
+    kc = synth.matrix(B * T, D, seed, synth.TENSOR_KC, "int").reshape(B, T, D)
+    w = synth.weights(B * S * H, seed, synth.TENSOR_W, "pow2").reshape(B, S, H)
+    return {"q": q, "kc": kc, "w": w}
+
+
+def _gauss_inputs(B, S, T, seed, H=64, D=128):
+    sig = 1 / np.sqrt(D)
+    q = synth.matrix(B * S * H, D, seed, synth.TENSOR_Q, "gauss", sig).reshape(B, S, H, D)
+    kc = synth.matrix(B * T, D, seed, synth.TENSOR_KC, "gauss", sig).reshape(B, T, D)
+    w = synth.weights(B * S * H, seed, synth.TENSOR_W, "uniform", 1 / np.sqrt(H)).reshape(B, S, H)
+    return {"q": q, "kc": kc, "w": w}
+
+
+# ---------------------------------------------------------------- exact cases
+@pytest.mark.parametrize("B,S,T,m,k,kw", [
+    (1, 256, 64, 4, 16, {}),                       # one diagonal tile, k < n
+    (1, 1024, 256, 4, 64, {}),                     # several key tiles
+    (1, 1027, 256, 4, 64, {}),                     # ragged query tail (S % 4 != 0)
+    (2, 512, 128, 4, 40, {}),                      # two sequences
+    (1, 600, 100, 4, 64, {}),                      # T < S/m: rows past 4T see all T keys
+    (1, 300, 200, 4, 64, {}),                      # T > S/m: trailing keys never visible
+    (1, 512, 512, 1, 100, {}),                     # m = 1
+    (1, 513, 171, 3, 37, {}),                      # m = 3, odd sizes
+    (1, 1024, 256, 4, 300, {}),                    # k > visible keys for most rows
+    (1, 1024, 256, 4, 1, {}),                      # k = 1
+    (1, 2048, 512, 4, 2048, {"key_tile": 128}),    # k = 2048 (max)
+    (1, 1024, 256, 4, 64, {"key_tile": 64}),       # 64-key partitions
+    (1, 2048, 512, 4, 64, {"key_tile": 1024}),     # 1024-key partitions
+    (1, 1024, 256, 4, 64, {"query_chunk": 256}),   # chunk driver, 4 launches
+    (1, 1020, 255, 4, 64, {"query_chunk": 100}),   # ragged chunks
+])
+def test_integer_inputs_bit_exact(B, S, T, m, k, kw):
+    inp = _int_inputs(B, S, T, seed=7 + S + T + k)
+    gi, gs = _run(inp, m, k, **kw)
+    rows = np.arange(B * S)
+    oi, osc, _ = oracle.topk(inp["q"], inp["kc"], inp["w"], m, k)
+    parity.check_structure(gi, gs, rows, S, T, m)
+    parity.compare_exact(gi, gs, oi, osc, rows)
+
+
+def test_all_zero_scores_return_first_indices():
+    inp = _int_inputs(1, 512, 128, seed=3)
+    inp["w"][:] = 0.0
+    gi, gs = _run(inp, 4, 32)
+    for t in range(512):
+        n = min(128, (t + 1) // 4)
+        want = np.full(32, -1)
+        want[: min(32, n)] = np.arange(min(32, n))
+        assert np.array_equal(gi[t], want), t
+        assert np.all(gs[t, : min(32, n)] == 0.0)
+
+
+def test_materialize_matches_oracle_exactly():
+    inp = _int_inputs(1, 1024, 256, seed=5)
+    gi, gs = _mat(inp, 4, 64)
+    oi, osc, _ = oracle.topk(inp["q"], inp["kc"], inp["w"], 4, 64)
+    parity.compare_exact(gi, gs, oi, osc, np.arange(1024))
+
+
+# ---------------------------------------------------------------- workloads
+def test_tiny_gaussian_workload():
+    wl = synth.WORKLOADS["tiny"]
+    inp = synth.make_inputs(wl)
+    gi, gs = _run(inp, wl.m, wl.k)
+    rows = np.arange(wl.S)
+    oi, _, osc64 = oracle.topk(inp["q"], inp["kc"], inp["w"], wl.m, wl.k)
+    parity.check_structure(gi, gs, rows, wl.S, wl.T, wl.m)
+    mean, mn = parity.compare_tolerant(gi, gs, oi, osc64, rows,
+                                       lambda r: oracle.scores(inp["q"], inp["kc"], inp["w"], wl.m, r))
+    assert mean >= parity.RECALL_MEAN and mn >= parity.RECALL_MIN, (mean, mn)
+    mi, ms = _mat(inp, wl.m, wl.k)
+    mean2, mn2 = parity.compare_tolerant(gi, gs, mi, ms.astype(np.float64), rows,
+                                         lambda r: oracle.scores(inp["q"], inp["kc"], inp["w"], wl.m, r))
+    assert mean2 >= parity.RECALL_MEAN and mn2 >= parity.RECALL_MIN
+
+
+def test_integer_workload_bit_exact():
+    """S=8192, k=512, integer inputs: streaming == oracle == materialize, bit for bit."""
+    wl = synth.WORKLOADS["integer"]
+    inp = synth.make_inputs(wl)
+    gi, gs = _run(inp, wl.m, wl.k)
+    rows = np.arange(wl.S)
+    oi, osc, _ = parity.oracle_rows("integer", rows, wl.k)
+    parity.check_structure(gi, gs, rows, wl.S, wl.T, wl.m)
+    parity.compare_exact(gi, gs, oi, osc, rows)
+    mi, ms = _mat(inp, wl.m, wl.k)
+    parity.compare_exact(mi, ms, oi, osc, rows)
+
+
+@pytest.fixture(scope="module")
+def sweep_oracle():
+    wl = synth.WORKLOADS["sweep"]
+    rows = np.arange(wl.S)
+    return parity.oracle_rows("sweep", rows, 1024)  # prefixes serve every k <= 1024
+
+
+@pytest.mark.parametrize("axis,value", [(a, v) for a in ("query_chunk", "key_tile", "k")
+                                        for v in synth.WORKLOADS["sweep"].sweep[a]])
+def test_design_space_sweep(axis, value, sweep_oracle):
+    wl = synth.WORKLOADS["sweep"]
+    inp = synth.make_inputs(wl)
+    k = value if axis == "k" else wl.k
+    kw = {axis: value} if axis != "k" else {}
+    gi, gs = _run(inp, wl.m, k, **kw)
+    rows = np.arange(wl.S)
+    oi, _, osc64 = (a[:, :k] for a in sweep_oracle)
+    parity.check_structure(gi, gs, rows, wl.S, wl.T, wl.m)
+    fn = lambda r: oracle.scores(inp["q"], inp["kc"], inp["w"], wl.m, r)  # noqa: E731
+    mean, mn = parity.compare_tolerant(gi, gs, oi, osc64, rows, fn)
+    assert mean >= parity.RECALL_MEAN and mn >= parity.RECALL_MIN, (axis, value, mean, mn)
+    mi, ms = _mat(inp, wl.m, k)
+    mean2, mn2 = parity.compare_tolerant(gi, gs, mi, ms.astype(np.float64), rows, fn)
+    assert mean2 >= parity.RECALL_MEAN and mn2 >= parity.RECALL_MIN, (axis, value, mean2, mn2)
+
+
+def _full_scores(inp, m, r, T, fmt):
+    """Oracle scores of every key of flat row r (NaN for invisible keys)."""
+    if fmt == "bf16":
+        return oracle.scores(inp["q"], inp["kc"], inp["w"], m, r)
+    ii, _, s64 = oracle.topk(inp["q"], inp["kc"], inp["w"], m, T, rows=[r],
+                             q_scale=inp["q_scale"], kc_scale=inp["kc_scale"])
+    full = np.full(T, np.nan)
+    v = ii[0] >= 0
+    full[ii[0][v]] = s64[0][v]
+    return full
+
+
+def _sampled(wl, gi, gs, inp, fmt="bf16"):
+    rows = synth.sample_rows(254, wl.m - 1, wl.S, seed=wl.seed)
+    first_full = wl.m * wl.k - 1  # first row with n >= k
+    rows = np.unique(np.concatenate([rows, [first_full, wl.S - 1]]))
+    oi, _, osc64 = parity.oracle_rows(wl.name, rows, wl.k, fmt=fmt)
+    parity.check_structure(gi[rows], gs[rows], rows, wl.S, wl.T, wl.m)
+
+    def fn(r):
+        return _full_scores(inp, wl.m, r, wl.T, fmt)
+
+    return parity.compare_tolerant(gi[rows], gs[rows], oi, osc64, rows, fn)
+
+
+def test_v4flash_sampled_rows():
+    """S=65536, k=512 planted-boost inputs; 256 sampled rows against the oracle."""
+    wl = synth.WORKLOADS["v4flash"]
+    inp = synth.make_inputs(wl)
+    gi, gs = _run(inp, wl.m, wl.k)
+    mean, mn = _sampled(wl, gi, gs, inp)
+    assert mean >= parity.RECALL_MEAN and mn >= parity.RECALL_MIN, (mean, mn)
+
+
+def test_materialize_refuses_v4flash_shape():
+    """The [1, 65536, 64, 16384] fp32 logits (256 GiB) exceed B200 memory: the
+    materialize path refuses with SI_ERR_OUT_OF_MEMORY instead of faulting."""
+    wl = synth.WORKLOADS["v4flash"]
+    q = torch.zeros((1, wl.S, wl.H, wl.D), dtype=torch.bfloat16, device="cuda")
+    kc = torch.zeros((1, wl.T, wl.D), dtype=torch.bfloat16, device="cuda")
+    w = torch.zeros((1, wl.S, wl.H), dtype=torch.float32, device="cuda")
+    with pytest.raises(si.SIError) as e:
+        si.indexer_materialize(q, kc, w, wl.m, wl.k)
+    assert e.value.status == si.SI_ERR_OUT_OF_MEMORY
+
+
+def test_bounded_wait_timeout_is_reported_and_context_survives():
+    inp = _int_inputs(1, 1024, 256, seed=11)
+    q, kc, w = _dev(inp)
+    out = torch.empty((1, 1024, 64), dtype=torch.int32, device="cuda")
+    assert si.test_stream_timeout(q, kc, w, 4, 64, out, wait_limit_ns=50_000_000) == si.SI_OK
+    assert si.device_status() == si.SI_ERR_TIMEOUT
+    assert si.device_status() == si.SI_OK  # record cleared
+    gi, gs = _run(inp, 4, 64)  # the context still works
+    oi, osc, _ = oracle.topk(inp["q"], inp["kc"], inp["w"], 4, 64)
+    parity.compare_exact(gi, gs, oi, osc, np.arange(1024))
+
+
+def test_unsupported_shapes_are_refused():
+    q = torch.zeros((1, 64, 32, 128), dtype=torch.bfloat16, device="cuda")
+    kc = torch.zeros((1, 16, 128), dtype=torch.bfloat16, device="cuda")
+    w = torch.zeros((1, 64, 32), dtype=torch.float32, device="cuda")
+    with pytest.raises(si.SIError) as e:
+        si.indexer_topk(q, kc, w, 4, 8)
+    assert e.value.status == si.SI_ERR_UNSUPPORTED
