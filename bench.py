@@ -278,7 +278,7 @@ def run_ours(args, wl):
     alg_bytes = q.numel() * 2 + kc.numel() * 2 + w.numel() * 4 + out_idx.numel() * 4 + out_score.numel() * 4
     traffic = ncu_traffic(wl.name)
     cpu = None
-    if world == 1:
+    if world == 1 and args.cpu_seconds > 0:
         rows = synth.sample_rows(4096, wl.m * 4, wl.S, seed=wl.seed + 99)
         rng = np.random.default_rng(wl.seed)
         rng.shuffle(rows)

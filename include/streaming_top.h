@@ -66,7 +66,7 @@ typedef struct si_options {
   int query_chunk;       /* queries per launch of the chunk driver; 0 = all S in one launch.
                             Must be a multiple of 4 otherwise. */
   int key_tile;          /* keys per partition of the partition-merge: 64 or a multiple
-                            of 128 up to 1024; 0 = 256 */
+                            of 128 up to 1024; 0 = 512 */
   void* workspace;       /* optional caller-owned device scratch, >= si_indexer_workspace_size() */
   size_t workspace_bytes;
 } si_options;

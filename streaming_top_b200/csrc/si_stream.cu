@@ -7,36 +7,46 @@
 //
 // One CTA per SM (persistent).  A work unit is a tile of QT = 4 consecutive
 // queries of one sequence; units are taken longest-first (the causal triangle
-// makes late queries see the most keys), dealt to CTAs in snake order.
+// makes late queries see the most keys) and dealt to CTAs in snake order.
 //
-// Per unit:
-//   warp 0 (one lane)  TMA: the unit's q tile [4 queries x 64 heads, 128]
-//                      (stationary) and then key tiles [128 keys, 128]
-//                      through an N-stage mbarrier ring, only the tiles
-//                      that hold a visible key.
-//   warp 1 (one lane)  tcgen05.mma, A = key tile (M = 128 keys), B = q tile
-//                      (N = 256 = 4 queries x 64 heads), K = 128, fp32
-//                      accumulator in TMEM, double buffered (2 x 256 columns)
-//                      so the MMA of tile j+1 overlaps the epilogue of tile j.
-//   warps 2..9         epilogue.  Thread = one key (TMEM lane), warp = 2 of
-//                      the 4 queries: tcgen05.ld of 64 head logits per query,
-//                      ReLU and w-weighted head sum in registers, causal mask,
-//                      then the partition-merge top-k:
-//                        - threshold early-reject: a key is appended to its
-//                          query's candidate pool only if its score beats the
-//                          k-th best score found at the last merge;
-//                        - at the end of every partition of `key_tile` keys
-//                          (the pages' key tile), a merge keeps exactly the k
-//                          best keys of the pool (radix select on the packed
-//                          key) and refreshes the threshold;
-//                        - at the end of the unit the k survivors are sorted
-//                          (bitonic, one warp per query) and stored.
+// Warp roles (16 warps):
+//   warp 0 (one lane)   TMA: the unit's q tile [4 queries x 64 heads, 128]
+//                       (stationary), then key tiles [128 keys, 128] through
+//                       an N-stage mbarrier ring -- only tiles holding a
+//                       visible key.
+//   warp 1 (one lane)   tcgen05.mma, A = key tile (M = 128 keys), B = q tile
+//                       (N = 256 = 4 queries x 64 heads), K = 128, fp32
+//                       accumulator in TMEM, double buffered (2 x 256
+//                       columns) so the MMA of tile j+1 overlaps the
+//                       epilogue of tile j.
+//   warps 8..15         scoring.  Warp = TMEM lane quadrant (warp % 4, 32
+//                       keys) x 2 of the 4 queries.  tcgen05.ld 16x256b gives
+//                       a thread 4 keys x 16 heads of a query; ReLU and the
+//                       w-weighted head sum run in registers (w held in
+//                       registers for the whole unit), a 2-step shuffle
+//                       reduce-scatter leaves each thread one key's score.
+//                       Causal mask, then threshold early-reject: a key is
+//                       appended to its query's candidate pool only if its
+//                       score beats the threshold the manager last
+//                       published; appends go to the warp's private segment
+//                       of a double-buffered append area.
+//   warps 4..7          top-k managers, one per query: they merge each
+//                       hand-off of candidates into the query's running pool
+//                       and count them into a 256-bin histogram of its
+//                       scores; at the end of every partition of `key_tile`
+//                       keys (the pages' key tile) they raise and publish
+//                       the threshold and compact the pool when it fills; at
+//                       the end of the unit they select the exact k best,
+//                       sort them and store them -- while the scoring warps
+//                       already work on the next unit.
+//   warps 2, 3          idle (they complete warpgroup 0).
 //
 // Keys are packed as (orderable fp32 score << 32) | ~index, so one unsigned
 // 64-bit comparison orders by score descending, then index ascending, and
-// every key is distinct.  Because key tiles are visited in index order, a new
-// key whose score merely ties the threshold has a larger index than the k-th
-// kept key and is correctly rejected: the filter needs the score only.
+// every key is distinct.  Because key tiles are visited in index order and a
+// threshold only ever comes from keys of earlier partitions, a new key whose
+// score merely ties the threshold has a larger index than the k-th kept key
+// and is correctly rejected: the filter needs the score only.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -45,21 +55,45 @@
 
 #include "si_internal.h"
 #include "si_ptx.cuh"
+#include "si_topk.cuh"
 
 namespace si {
 namespace {
 
-constexpr int QT = 4;          // queries per unit
-constexpr int HEADS = 64;      // indexer heads (H_I)
-constexpr int DIM = 128;       // head dim (D)
-constexpr int KT = 128;        // keys per MMA tile (M)
+constexpr int QT = 4;              // queries per unit
+constexpr int HEADS = 64;          // indexer heads (H_I)
+constexpr int DIM = 128;           // head dim (D)
+constexpr int KT = 128;            // keys per MMA tile (M)
 constexpr int NCOLS = QT * HEADS;  // 256 = MMA N
-constexpr int THREADS = 320;   // 10 warps
-constexpr int EPI_THREADS = 256;
+constexpr int THREADS = 512;       // 16 warps
+constexpr int N_SCORE_WARPS = 8;
 constexpr int HIST_BINS = 256;
+constexpr int N_AREAS = 2;         // append areas (double buffered)
+constexpr int CTRL_BYTES = 1024;
+// Register budgets: launched at 128 per thread (512 threads); warpgroup 0
+// (producer, MMA) and warpgroup 1 (managers) give registers to the two
+// scoring warpgroups: 128 * 40 + 128 * 120 + 256 * 176 = 65536.
+constexpr uint32_t REGS_PIPE = 40;
+constexpr uint32_t REGS_MGR = 120;
+constexpr uint32_t REGS_SCORE = 176;
+static_assert(128 * REGS_PIPE + 128 * REGS_MGR + 256 * REGS_SCORE <= 512 * 128, "register split");
+
+// Scoring warps hand their candidates to the managers in sub-partitions of
+// at most 256 keys (a 64-key partition is half a tile, otherwise 1 or 2
+// tiles); the managers refresh the threshold once per partition.
+__host__ __device__ constexpr int sub_keys(int key_tile) {
+  return key_tile <= 256 ? key_tile : (key_tile % 256 == 0 ? 256 : 128);
+}
+__host__ __device__ constexpr int sub_tiles(int key_tile) {
+  return sub_keys(key_tile) >= KT ? sub_keys(key_tile) / KT : 1;
+}
+// Appends one scoring warp can make to one query's pool in one
+// sub-partition: 32 keys per 128-key tile.
+__host__ __device__ constexpr int seg_capacity(int key_tile) { return 32 * sub_tiles(key_tile); }
 
 enum { ERR_WAIT_Q = 1, ERR_WAIT_KC = 2, ERR_WAIT_TMEM_EMPTY = 3, ERR_WAIT_TMEM_FULL = 4,
-       ERR_WAIT_QFREE = 5, ERR_WAIT_KFREE = 6, ERR_WAIT_DRAIN = 7 };
+       ERR_WAIT_QFREE = 5, ERR_WAIT_KFREE = 6, ERR_WAIT_DRAIN = 7, ERR_WAIT_SEG_FREE = 8,
+       ERR_WAIT_SEG_DONE = 9 };
 
 struct Params {
   const float* w;         // [B,S,H]
@@ -71,7 +105,7 @@ struct Params {
   int B, S, T, m, k;
   int qt_begin, qt_end;   // query tiles (per sequence) of this launch
   int key_tile;           // partition length in keys (64 or multiple of 128)
-  int pool_cap;           // pool entries per query
+  int cap;                // main-region entries per query pool
   int n_stages;
   uint64_t wait_limit_ns;
   int test_withhold;
@@ -102,15 +136,16 @@ __device__ __forceinline__ int unit_of(int i, int n_units) {
   return u < n_units ? static_cast<int>(u) : -1;
 }
 
+__device__ __forceinline__ int n_subparts(const Unit& U, const Params& p) {
+  if (p.key_tile < KT) return 2 * U.n_kt;
+  const int st = sub_tiles(p.key_tile);
+  return (U.n_kt + st - 1) / st;
+}
+
 __device__ __forceinline__ uint32_t f32_ord(float f) {
   uint32_t u = __float_as_uint(f);
   if (u == 0x80000000u) u = 0u;  // -0 ranks with +0
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
-__device__ __forceinline__ float ord_f32(uint32_t o) {
-  const uint32_t u = (o & 0x80000000u) ? (o & 0x7FFFFFFFu) : ~o;
-  return __uint_as_float(u);
 }
 
 __device__ __forceinline__ void record_error(const Params& p, volatile int* abort, int where) {
@@ -119,182 +154,98 @@ __device__ __forceinline__ void record_error(const Params& p, volatile int* abor
   *abort = 1;
 }
 
-__device__ __forceinline__ void epi_sync() {
-  asm volatile("bar.sync 1, %0;" ::"n"(EPI_THREADS) : "memory");
+// Packed fp32 pair FMA (sm_100): d = a * b + d on two lanes of a 64-bit register.
+__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %5};\n\t"
+      "mov.b64 rd, {%0, %1};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rd;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "+f"(d0), "+f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
-__device__ __forceinline__ uint64_t shfl_xor_u64(uint64_t v, int m) {
-  const uint32_t lo = __shfl_xor_sync(0xFFFFFFFFu, static_cast<uint32_t>(v), m);
-  const uint32_t hi = __shfl_xor_sync(0xFFFFFFFFu, static_cast<uint32_t>(v >> 32), m);
-  return (static_cast<uint64_t>(hi) << 32) | lo;
-}
+__device__ __forceinline__ float relu_u(uint32_t x) { return fmaxf(__uint_as_float(x), 0.f); }
 
-// Merge step of the partition-merge top-k, one warp: keep exactly the k
-// largest packed keys of pool[0, n) (n > k), in place, and return the
-// threshold (orderable score of the k-th key).  Radix select, most
-// significant digit first, starting below the bits all keys share.
-__device__ uint32_t pool_shrink(uint64_t* pool, int n, int k, uint32_t* hist, int lane) {
-  uint64_t vor = 0, vand = ~0ull;
-  for (int i = lane; i < n; i += 32) {
-    const uint64_t x = pool[i];
-    vor |= x;
-    vand &= x;
-  }
+// One query's scores for the thread's key.  va / vb: 16x256b.x8 loads of the
+// quadrant's lanes 0-15 and 16-31: register 4r+e holds (key t1, head
+// 8r+2t0+e), register 4r+2+e holds (key t1+8, same head), where t0 = lane%4,
+// t1 = lane/4; vb likewise for keys t1+16, t1+24.  wq[2r+e] = w of head
+// 8r+2t0+e.  The four lanes sharing t1 reduce-scatter their 16-head partial
+// sums so that lane t0 ends with the full sum of key t1 + 8*t0.
+__device__ __forceinline__ float score_query(const uint32_t (&va)[32], const uint32_t (&vb)[32],
+                                             const float (&wq)[16], int lane) {
+  float s[4][2];
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    vor |= shfl_xor_u64(vor, o);
-    vand &= shfl_xor_u64(vand, o);
-  }
-  const uint64_t diff = vor ^ vand;  // non-zero: keys are distinct and n >= 2
-  const int hb = 63 - __clzll(static_cast<long long>(diff));
-  uint64_t mask = hb == 63 ? 0ull : (~0ull << (hb + 1));
-  uint64_t prefix = vand & mask;
-  int need = k;
-  int hi = hb + 1;
-  for (;;) {
-    const int lo = hi > 8 ? hi - 8 : 0;
-    const uint32_t dmask = (1u << (hi - lo)) - 1u;
-    for (int i = lane; i < HIST_BINS; i += 32) hist[i] = 0u;
-    __syncwarp();
-    for (int i = lane; i < n; i += 32) {
-      const uint64_t x = pool[i];
-      if ((x & mask) == prefix) atomicAdd(&hist[static_cast<uint32_t>(x >> lo) & dmask], 1u);
-    }
-    __syncwarp();
-    // lane l owns digits 255-8l .. 248-8l (descending)
-    uint32_t c[8], sum = 0;
+  for (int j = 0; j < 4; ++j) s[j][0] = s[j][1] = 0.f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      c[i] = hist[255 - 8 * lane - i];
-      sum += c[i];
-    }
-    uint32_t incl = sum;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-      if (lane >= o) incl += v;
-    }
-    const uint32_t excl = incl - sum;
-    const bool mine = excl < static_cast<uint32_t>(need) && static_cast<uint32_t>(need) <= incl;
-    const uint32_t owners = __ballot_sync(0xFFFFFFFFu, mine);
-    const int owner = __ffs(owners) - 1;
-    int d = 0;
-    uint32_t above = 0, cd = 0;
-    if (lane == owner) {
-      uint32_t run = excl;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        if (run + c[i] >= static_cast<uint32_t>(need)) {
-          d = 255 - 8 * lane - i;
-          above = run;
-          cd = c[i];
-          break;
-        }
-        run += c[i];
-      }
-    }
-    d = __shfl_sync(0xFFFFFFFFu, d, owner);
-    above = __shfl_sync(0xFFFFFFFFu, above, owner);
-    cd = __shfl_sync(0xFFFFFFFFu, cd, owner);
-    need -= static_cast<int>(above);
-    prefix |= static_cast<uint64_t>(d) << lo;
-    mask |= static_cast<uint64_t>(dmask) << lo;
-    __syncwarp();
-    if (cd == static_cast<uint32_t>(need) || lo == 0) break;
-    hi = lo;
+  for (int r = 0; r < 8; ++r) {
+    const float w0 = wq[2 * r], w1 = wq[2 * r + 1];
+    fma2(s[0][0], s[0][1], w0, w1, relu_u(va[4 * r + 0]), relu_u(va[4 * r + 1]));
+    fma2(s[1][0], s[1][1], w0, w1, relu_u(va[4 * r + 2]), relu_u(va[4 * r + 3]));
+    fma2(s[2][0], s[2][1], w0, w1, relu_u(vb[4 * r + 0]), relu_u(vb[4 * r + 1]));
+    fma2(s[3][0], s[3][1], w0, w1, relu_u(vb[4 * r + 2]), relu_u(vb[4 * r + 3]));
   }
-  // keep the keys whose leading bits are >= prefix: exactly k of them
-  int kept = 0;
-  uint64_t kmin = ~0ull;
-  for (int base = 0; base < n; base += 32) {
-    const int i = base + lane;
-    const uint64_t x = i < n ? pool[i] : 0ull;
-    const bool keep = i < n && (x & mask) >= prefix;
-    const uint32_t bal = __ballot_sync(0xFFFFFFFFu, keep);
-    __syncwarp();
-    if (keep) {
-      pool[kept + __popc(bal & ((1u << lane) - 1u))] = x;
-      kmin = x < kmin ? x : kmin;
-    }
-    kept += __popc(bal);
-    __syncwarp();
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const uint64_t y = shfl_xor_u64(kmin, o);
-    kmin = y < kmin ? y : kmin;
-  }
-  return static_cast<uint32_t>(kmin >> 32);
-}
-
-// Bitonic sort of a[0, np) into descending order, one warp (np power of two).
-__device__ void warp_sort_desc(uint64_t* a, int np, int lane) {
-  for (int size = 2; size <= np; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = lane; i < (np >> 1); i += 32) {
-        const int lo = 2 * i - (i & (stride - 1));
-        const int hi = lo + stride;
-        const bool desc = (lo & size) == 0;
-        const uint64_t x = a[lo], y = a[hi];
-        if ((x < y) == desc) {
-          a[lo] = y;
-          a[hi] = x;
-        }
-      }
-      __syncwarp();
-    }
-  }
-}
-
-// sum_h w[h] * ReLU(L[h]) over the 64 head logits of one (key, query) pair,
-// held as two 32-column TMEM loads; four partial sums for ILP.
-__device__ __forceinline__ float head_sum(const uint32_t (&lo)[32], const uint32_t (&hi)[32],
-                                          const float* w) {
-  const float4* w4 = reinterpret_cast<const float4*>(w);
-  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll
-  for (int h = 0; h < 32; h += 4) {
-    const float4 ww = w4[h >> 2];
-    a0 = fmaf(ww.x, fmaxf(__uint_as_float(lo[h + 0]), 0.f), a0);
-    a1 = fmaf(ww.y, fmaxf(__uint_as_float(lo[h + 1]), 0.f), a1);
-    a2 = fmaf(ww.z, fmaxf(__uint_as_float(lo[h + 2]), 0.f), a2);
-    a3 = fmaf(ww.w, fmaxf(__uint_as_float(lo[h + 3]), 0.f), a3);
-  }
-#pragma unroll
-  for (int h = 0; h < 32; h += 4) {
-    const float4 ww = w4[8 + (h >> 2)];
-    a0 = fmaf(ww.x, fmaxf(__uint_as_float(hi[h + 0]), 0.f), a0);
-    a1 = fmaf(ww.y, fmaxf(__uint_as_float(hi[h + 1]), 0.f), a1);
-    a2 = fmaf(ww.z, fmaxf(__uint_as_float(hi[h + 2]), 0.f), a2);
-    a3 = fmaf(ww.w, fmaxf(__uint_as_float(hi[h + 3]), 0.f), a3);
-  }
-  return (a0 + a1) + (a2 + a3);
+  const float p0 = s[0][0] + s[0][1], p1 = s[1][0] + s[1][1];
+  const float p2 = s[2][0] + s[2][1], p3 = s[3][0] + s[3][1];
+  const bool b0 = lane & 1, b1 = (lane >> 1) & 1;
+  // step 1: keep keys {b0, b0 + 2}, hand the other two to lane ^ 1
+  const float k0 = b0 ? p1 : p0, k1 = b0 ? p3 : p2;
+  const float g0 = b0 ? p0 : p1, g1 = b0 ? p2 : p3;
+  const float r0 = k0 + __shfl_xor_sync(0xFFFFFFFFu, g0, 1);
+  const float r1 = k1 + __shfl_xor_sync(0xFFFFFFFFu, g1, 1);
+  // step 2: keep key b0 + 2*b1
+  const float keep = b1 ? r1 : r0, give = b1 ? r0 : r1;
+  return keep + __shfl_xor_sync(0xFFFFFFFFu, give, 2);
 }
 
 // Shared-memory layout (offsets from a 1024-byte aligned base).
 template <int OPB>
 struct Layout {
-  static constexpr int Q_HALF = NCOLS * 128;               // bytes per 128-byte-wide K column block of q
-  static constexpr int Q_BYTES = NCOLS * DIM * OPB;        // 64 KB bf16, 32 KB fp8
+  static constexpr int Q_HALF = NCOLS * 128;         // one 128-byte-wide K column block of q
+  static constexpr int Q_BYTES = NCOLS * DIM * OPB;  // 64 KB bf16, 32 KB fp8
   static constexpr int KC_HALF = KT * 128;
-  static constexpr int KC_BYTES = KT * DIM * OPB;          // 32 KB bf16, 16 KB fp8
-  static constexpr int N_MMA = DIM * OPB / 32;             // K steps of 32 bytes
+  static constexpr int KC_BYTES = KT * DIM * OPB;    // 32 KB bf16, 16 KB fp8
+  static constexpr int N_MMA = DIM * OPB / 32;       // K steps of 32 bytes
 };
+
+// Per-query pool: main region [0, cap) then N_AREAS append areas of
+// 4 * seg_cap entries each.
+__host__ __device__ constexpr int pool_stride(int cap, int seg_cap) {
+  return cap + N_AREAS * 4 * seg_cap;
+}
 
 struct Smem {
-  uint32_t q, kc, pool, w, hist, ctrl;
+  uint32_t q, kc, pool, hist, ctrl;
 };
 
-__device__ __forceinline__ Smem carve(int n_stages, int pool_cap, int q_bytes, int kc_bytes) {
+__host__ __device__ inline Smem carve(int n_stages, int cap, int seg_cap, int q_bytes, int kc_bytes) {
   Smem s;
   s.q = 0;
   s.kc = q_bytes;
   s.pool = s.kc + n_stages * kc_bytes;
-  s.w = s.pool + QT * pool_cap * 8;
-  s.hist = s.w + QT * HEADS * 4;
+  s.hist = s.pool + QT * pool_stride(cap, seg_cap) * 8;
   s.ctrl = s.hist + QT * HIST_BINS * 4;
   return s;
 }
+
+// Control block (CTRL_BYTES): mbarriers, manager state, published
+// thresholds, segment counts, TMEM slot, abort flag.
+struct Ctrl {
+  uint64_t full[4], empty[4];
+  uint64_t q_full, q_empty;
+  uint64_t t_full[2], t_empty[2];
+  uint64_t mma_done;
+  uint64_t seg_done[N_AREAS][2];  // [area][query pair]: scoring warps -> manager
+  uint64_t seg_free[N_AREAS][2];  // manager -> scoring warps
+  uint64_t pub[QT];               // (unit tag << 32) | threshold
+  topk::QState qs[QT];
+  uint32_t seg_cnt[N_AREAS][QT][4];
+  uint32_t tmem_slot;
+  int abort;
+};
+static_assert(sizeof(Ctrl) <= CTRL_BYTES, "control block");
 
 template <int OPB>
 __global__ void __launch_bounds__(THREADS, 1)
@@ -304,39 +255,36 @@ __global__ void __launch_bounds__(THREADS, 1)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  const Smem so = carve(p.n_stages, p.pool_cap, L::Q_BYTES, L::KC_BYTES);
+  const int seg_cap = seg_capacity(p.key_tile);
+  const int stride = pool_stride(p.cap, seg_cap);
+  const Smem so = carve(p.n_stages, p.cap, seg_cap, L::Q_BYTES, L::KC_BYTES);
   uint8_t* q_s = smem + so.q;
   uint8_t* kc_s = smem + so.kc;
-  uint64_t* pool = reinterpret_cast<uint64_t*>(smem + so.pool);
-  float* w_s = reinterpret_cast<float*>(smem + so.w);
+  uint64_t* pools = reinterpret_cast<uint64_t*>(smem + so.pool);
   uint32_t* hist = reinterpret_cast<uint32_t*>(smem + so.hist);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + so.ctrl);
-  uint64_t* full = bars;                        // [n_stages]
-  uint64_t* empty = bars + 4;                   // [n_stages]
-  uint64_t* q_full = bars + 8;
-  uint64_t* q_empty = bars + 9;
-  uint64_t* t_full = bars + 10;                 // [2]
-  uint64_t* t_empty = bars + 12;                // [2]
-  uint64_t* mma_done = bars + 14;
-  uint32_t* cnt = reinterpret_cast<uint32_t*>(bars + 16);  // [QT]
-  uint32_t* thr = cnt + QT;                                // [QT]
-  uint32_t* tmem_slot = thr + QT;
-  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  Ctrl* C = reinterpret_cast<Ctrl*>(smem + so.ctrl);
+  volatile int* abort = &C->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.n_stages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&C->full[s], 1);
+      mbar_init(&C->empty[s], 1);
     }
-    mbar_init(q_full, 1);
-    mbar_init(q_empty, 1);
+    mbar_init(&C->q_full, 1);
+    mbar_init(&C->q_empty, 1);
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&t_full[b], 1);
-      mbar_init(&t_empty[b], 8);  // one arrival per epilogue warp
+      mbar_init(&C->t_full[b], 1);
+      mbar_init(&C->t_empty[b], N_SCORE_WARPS);
     }
-    mbar_init(mma_done, 1);
+    mbar_init(&C->mma_done, 1);
+    for (int a = 0; a < N_AREAS; ++a)
+      for (int g = 0; g < 2; ++g) {
+        mbar_init(&C->seg_done[a][g], 4);  // the 4 scoring warps of a query pair
+        mbar_init(&C->seg_free[a][g], 2);  // the pair's two managers
+      }
+    for (int q = 0; q < QT; ++q) C->pub[q] = 0ull;
     *abort = 0;
     fence_mbar_init();
   }
@@ -344,18 +292,19 @@ __global__ void __launch_bounds__(THREADS, 1)
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_kc);
   }
-  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  if (warp == 1) tmem_alloc(&C->tmem_slot, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem = C->tmem_slot;
 
   const int n_units = p.B * (p.qt_end - p.qt_begin);
   const int q_bytes = L::Q_BYTES, kc_bytes = L::KC_BYTES;
 
-  if (warp == 0) {
+  if (warp < 4) {
+    regs_dec<REGS_PIPE>();
+    if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
       uint32_t stage = 0, phase = 0, qph = 0;
       uint32_t any_load = 0, last_par = 0;  // per stage bit: loaded at all / parity of last load
       uint32_t q_issued = 0;
@@ -365,29 +314,31 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (u < 0 || *abort) break;
         const Unit U = decode_unit(u, p);
         if (U.n_kt == 0) continue;
-        if (!mbar_wait_bounded(q_empty, qph ^ 1u, abort, p.wait_limit_ns)) {
+        if (!mbar_wait_bounded(&C->q_empty, qph ^ 1u, abort, p.wait_limit_ns)) {
           record_error(p, abort, ERR_WAIT_QFREE);
           break;
         }
-        mbar_arrive_expect_tx(q_full, q_bytes);
+        mbar_arrive_expect_tx(&C->q_full, q_bytes);
         const int qrow = (U.b * p.S + U.t0) * HEADS;
-        for (int h = 0; h < OPB; ++h) tma_load_2d(q_s + h * L::Q_HALF, &tm_q, q_full, h * (128 / OPB), qrow);
+        for (int h = 0; h < OPB; ++h)
+          tma_load_2d(q_s + h * L::Q_HALF, &tm_q, &C->q_full, h * (128 / OPB), qrow);
         ++q_issued;
         qph ^= 1u;
         bool stop = false;
         for (int j = 0; j < U.n_kt; ++j) {
-          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort, p.wait_limit_ns)) {
+          if (!mbar_wait_bounded(&C->empty[stage], phase ^ 1u, abort, p.wait_limit_ns)) {
             record_error(p, abort, ERR_WAIT_KFREE);
             stop = true;
             break;
           }
-          mbar_arrive_expect_tx(&full[stage], kc_bytes);
+          mbar_arrive_expect_tx(&C->full[stage], kc_bytes);
           const int krow = U.b * p.T + j * KT;
           if (p.test_withhold && !withheld && blockIdx.x == 0) {
             withheld = true;  // test hook: never deliver this tile
           } else {
             uint8_t* dst = kc_s + stage * kc_bytes;
-            for (int h = 0; h < OPB; ++h) tma_load_2d(dst + h * L::KC_HALF, &tm_kc, &full[stage], h * (128 / OPB), krow);
+            for (int h = 0; h < OPB; ++h)
+              tma_load_2d(dst + h * L::KC_HALF, &tm_kc, &C->full[stage], h * (128 / OPB), krow);
             any_load |= 1u << stage;
             last_par = (last_par & ~(1u << stage)) | (phase << stage);
           }
@@ -401,15 +352,13 @@ __global__ void __launch_bounds__(THREADS, 1)
       // drain: the last real load of every stage has landed before exit
       for (int s = 0; s < p.n_stages; ++s) {
         if (!((any_load >> s) & 1u)) continue;
-        if (!mbar_wait_timed(&full[s], (last_par >> s) & 1u, p.wait_limit_ns))
+        if (!mbar_wait_timed(&C->full[s], (last_par >> s) & 1u, p.wait_limit_ns))
           record_error(p, abort, ERR_WAIT_DRAIN);
       }
-      if (q_issued && !mbar_wait_timed(q_full, (q_issued - 1) & 1u, p.wait_limit_ns))
+      if (q_issued && !mbar_wait_timed(&C->q_full, (q_issued - 1) & 1u, p.wait_limit_ns))
         record_error(p, abort, ERR_WAIT_DRAIN);
-    }
-  } else if (warp == 1) {
+    } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
       constexpr uint32_t IDESC = OPB == 2 ? idesc_f32acc(1, 1, KT, NCOLS) : idesc_f32acc(0, 0, KT, NCOLS);
       const uint32_t q_addr = smem_u32(q_s), kc_addr = smem_u32(kc_s);
       uint32_t stage = 0, phase = 0, qph = 0, acc = 0, accph = 0;
@@ -418,7 +367,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (u < 0 || *abort) break;
         const Unit U = decode_unit(u, p);
         if (U.n_kt == 0) continue;
-        if (!mbar_wait_bounded(q_full, qph, abort, p.wait_limit_ns)) {
+        if (!mbar_wait_bounded(&C->q_full, qph, abort, p.wait_limit_ns)) {
           record_error(p, abort, ERR_WAIT_Q);
           break;
         }
@@ -426,12 +375,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_after();
         bool stop = false;
         for (int j = 0; j < U.n_kt; ++j) {
-          if (!mbar_wait_bounded(&t_empty[acc], accph ^ 1u, abort, p.wait_limit_ns)) {
+          if (!mbar_wait_bounded(&C->t_empty[acc], accph ^ 1u, abort, p.wait_limit_ns)) {
             record_error(p, abort, ERR_WAIT_TMEM_EMPTY);
             stop = true;
             break;
           }
-          if (!mbar_wait_bounded(&full[stage], phase, abort, p.wait_limit_ns)) {
+          if (!mbar_wait_bounded(&C->full[stage], phase, abort, p.wait_limit_ns)) {
             record_error(p, abort, ERR_WAIT_KC);
             stop = true;
             break;
@@ -449,9 +398,9 @@ __global__ void __launch_bounds__(THREADS, 1)
             else
               mma_f8(d_tmem, sdesc_kmajor_sw128(a0 + aoff), sdesc_kmajor_sw128(q_addr + boff), IDESC, kk > 0);
           }
-          mma_commit(&empty[stage]);
-          mma_commit(&t_full[acc]);
-          if (j == U.n_kt - 1) mma_commit(q_empty);
+          mma_commit(&C->empty[stage]);
+          mma_commit(&C->t_full[acc]);
+          if (j == U.n_kt - 1) mma_commit(&C->q_empty);
           if (++stage == static_cast<uint32_t>(p.n_stages)) {
             stage = 0;
             phase ^= 1u;
@@ -464,140 +413,177 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (stop) break;
       }
       // every MMA issued above has completed before TMEM is released
-      mma_commit(mma_done);
-      if (!mbar_wait_timed(mma_done, 0, p.wait_limit_ns)) record_error(p, abort, ERR_WAIT_DRAIN);
+      mma_commit(&C->mma_done);
+      if (!mbar_wait_timed(&C->mma_done, 0, p.wait_limit_ns)) record_error(p, abort, ERR_WAIT_DRAIN);
     }
-  } else {
-    // ------------------------------------------------------------ epilogue
-    const int etid = threadIdx.x - 64;  // 0..255
-    const int ew = warp - 2;            // 0..7
-    const int quad = warp & 3;          // TMEM lanes 32*quad .. 32*quad+31
-    const int qp = ew >> 2;             // this warp's queries: 2*qp, 2*qp+1
+  } else if (warp < 8) {
+    regs_dec<REGS_MGR>();
+    // ------------------------------------------------------------ top-k managers
+    const int q = warp - 4;   // this manager's query in the unit
+    const int g = q >> 1;     // the query pair whose scoring warps feed it
     const int k = p.k;
-    const bool half_parts = p.key_tile < KT;
-    const int part_tiles = half_parts ? 1 : p.key_tile / KT;
-    uint32_t acc = 0, accph = 0;
+    const int room = p.key_tile;  // appends one partition can bring
+    const int subs_per_part = p.key_tile / sub_keys(p.key_tile);
+    uint64_t* pool = pools + q * stride;
+    uint32_t* qh = hist + q * HIST_BINS;
+    topk::QState* st = &C->qs[q];
+    uint32_t gp = 0;          // hand-offs merged so far (CTA-wide numbering)
+    bool ok = true;
     for (int i = 0;; ++i) {
       const int u = unit_of(i, n_units);
       if (u < 0) break;
       const Unit U = decode_unit(u, p);
-      const bool live = !*abort;
-      {
-        const int q = etid >> 6, h = etid & 63, t = U.t0 + q;
-        float wv = 0.f;
-        if (t < p.S) {
-          const size_t wi = (static_cast<size_t>(U.b) * p.S + t) * HEADS + h;
-          wv = p.w[wi];
-          if (OPB == 1) wv *= p.q_scale[wi];
-        }
-        w_s[q * HEADS + h] = wv;
-        if (etid < QT) {
-          cnt[etid] = 0;
-          thr[etid] = 0;
-        }
+      if (lane == 0) {
+        st->cnt = 0;
+        st->thr = 0;
+        st->base = 0;
+        st->shift = 0;
+        st->binned = 0;
       }
+      __syncwarp();
+      const int np = n_subparts(U, p);
+      for (int pi = 0; pi < np; ++pi, ++gp) {
+        const int a = gp & 1;
+        const uint32_t use = gp >> 1;
+        if (ok && !*abort && !mbar_wait_bounded(&C->seg_done[a][g], use & 1u, abort, p.wait_limit_ns)) {
+          record_error(p, abort, ERR_WAIT_SEG_DONE);
+          ok = false;
+        }
+        ok = ok && !*abort;
+        if (ok) {
+          topk::merge(st, pool, pool + p.cap + a * 4 * seg_cap, C->seg_cnt[a][q], seg_cap, qh, lane);
+          if (((pi + 1) % subs_per_part == 0) || (pi == np - 1)) {
+            topk::refresh(st, pool, qh, k, p.cap, room, lane);
+            if (lane == 0)
+              *reinterpret_cast<volatile uint64_t*>(&C->pub[q]) = (static_cast<uint64_t>(i) << 32) | st->thr;
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&C->seg_free[a][g]);
+      }
+      // finalize this unit's query while the scorers move on
+      const int t = U.t0 + q;
+      if (t < p.S) {
+        if (!ok && lane == 0) st->cnt = 0;  // after an abort: contents unspecified
+        __syncwarp();
+        const size_t ob = (static_cast<size_t>(U.b) * p.S + t) * static_cast<size_t>(k);
+        topk::finalize(st, pool, qh, k, p.out_idx + ob, p.out_score ? p.out_score + ob : nullptr, lane);
+      }
+    }
+  } else {
+    regs_inc<REGS_SCORE>();
+    // ------------------------------------------------------------ scoring warps
+    const int quad = warp & 3;        // TMEM lanes 32*quad .. 32*quad+31
+    const int qp = (warp - 8) >> 2;   // this warp's queries: 2*qp, 2*qp+1
+    const int t0 = lane & 3, t1 = lane >> 2;
+    const int key_off = quad * 32 + t1 + 8 * t0;  // key (within the tile) this lane scores
+    const bool half_parts = p.key_tile < KT;
+    const int part_tiles = sub_tiles(p.key_tile);  // tiles per hand-off
+    const int n_phase = half_parts ? 2 : 1;
+    uint32_t acc = 0, accph = 0, gp = 0;
+    for (int i = 0;; ++i) {
+      const int u = unit_of(i, n_units);
+      if (u < 0) break;
+      const Unit U = decode_unit(u, p);
+      if (U.n_kt == 0) continue;
+      // w of this lane's 16 heads (8r + 2*t0 + e) for both queries
+      float wq[2][16];
       int nvis[2];
 #pragma unroll
       for (int qi = 0; qi < 2; ++qi) {
         const int t = U.t0 + 2 * qp + qi;
         const int n = t < p.S ? (t + 1) / p.m : 0;
         nvis[qi] = n < p.T ? n : p.T;
+        const size_t wb = (static_cast<size_t>(U.b) * p.S + (t < p.S ? t : p.S - 1)) * HEADS;
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int h = 8 * r + 2 * t0 + e;
+            float wv = p.w[wb + h];
+            if (OPB == 1) wv *= p.q_scale[wb + h];
+            wq[qi][2 * r + e] = t < p.S ? wv : 0.f;
+          }
+        }
       }
-      epi_sync();
+      uint32_t thr_r[2] = {0u, 0u};
+      uint32_t seg_n[2] = {0u, 0u};
+      uint64_t* seg_ptr[2] = {pools, pools};
+      bool ok = !*abort;
       for (int j = 0; j < U.n_kt; ++j) {
-        bool ok = live && !*abort;
-        if (ok && !mbar_wait_bounded(&t_full[acc], accph, abort, p.wait_limit_ns)) {
+        ok = ok && !*abort;
+        if (ok && !mbar_wait_bounded(&C->t_full[acc], accph, abort, p.wait_limit_ns)) {
           record_error(p, abort, ERR_WAIT_TMEM_FULL);
           ok = false;
         }
-        const int s = j * KT + quad * 32 + lane;
-        uint64_t key[2] = {0ull, 0ull};
-        bool pass[2] = {false, false};
+        const int s = j * KT + key_off;
+        uint32_t ord[2] = {0u, 0u};
         if (ok) {
           tc_fence_after();
-          const uint32_t ta =
-              tmem + (static_cast<uint32_t>(quad * 32) << 16) + acc * NCOLS + (2 * qp) * HEADS;
+          const uint32_t ta = tmem + (static_cast<uint32_t>(quad * 32) << 16) + acc * NCOLS + (2 * qp) * HEADS;
           float ksc = 1.f;
           if (OPB == 1 && s < p.T) ksc = p.kc_scale[static_cast<size_t>(U.b) * p.T + s];
-          float sc[2];
 #pragma unroll
           for (int qi = 0; qi < 2; ++qi) {
-            uint32_t v0[32], v1[32];
-            tmem_ld32(ta + qi * HEADS, v0);
-            tmem_ld32(ta + qi * HEADS + 32, v1);
+            uint32_t va[32], vb[32];
+            tmem_ld_16x256b_x8(ta + qi * HEADS, va);
+            tmem_ld_16x256b_x8(ta + (16u << 16) + qi * HEADS, vb);
             tmem_ld_wait();
-            sc[qi] = head_sum(v0, v1, w_s + (2 * qp + qi) * HEADS) * ksc;
+            ord[qi] = f32_ord(score_query(va, vb, wq[qi], lane) * ksc);
           }
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&t_empty[acc]);  // accumulator may be overwritten now
-          const float s0 = sc[0], s1 = sc[1];
-          key[0] = (static_cast<uint64_t>(f32_ord(s0)) << 32) | static_cast<uint32_t>(~static_cast<uint32_t>(s));
-          key[1] = (static_cast<uint64_t>(f32_ord(s1)) << 32) | static_cast<uint32_t>(~static_cast<uint32_t>(s));
-          pass[0] = s < nvis[0];
-          pass[1] = s < nvis[1];
+          if (lane == 0) mbar_arrive(&C->t_empty[acc]);  // accumulator may be overwritten now
+#pragma unroll
+          for (int qi = 0; qi < 2; ++qi) {  // adopt the manager's latest threshold for this unit
+            const uint64_t pv = *reinterpret_cast<volatile uint64_t*>(&C->pub[2 * qp + qi]);
+            if (static_cast<int>(pv >> 32) == i) thr_r[qi] = max(thr_r[qi], static_cast<uint32_t>(pv));
+          }
         }
         if (++acc == 2) {
           acc = 0;
           accph ^= 1u;
         }
-        // append survivors of the threshold; with 64-key partitions the two
-        // halves of the tile are separate partitions (merge in between)
-        const int n_phase = half_parts ? 2 : 1;
+        const uint32_t low = static_cast<uint32_t>(~static_cast<uint32_t>(s));
         for (int ph = 0; ph < n_phase; ++ph) {
-          const bool mine = !half_parts || (quad >> 1) == ph;
-          if (mine) {
+          const int a = gp & 1;
+          const bool starts = half_parts || (j % part_tiles == 0);
+          if (starts) {
+            // open an append area: wait until its manager has merged its last use
+            const uint32_t use = gp >> 1;
+            if (ok && !mbar_wait_bounded(&C->seg_free[a][qp], (use & 1u) ^ 1u, abort, p.wait_limit_ns)) {
+              record_error(p, abort, ERR_WAIT_SEG_FREE);
+              ok = false;
+            }
 #pragma unroll
             for (int qi = 0; qi < 2; ++qi) {
-              const int q = 2 * qp + qi;
-              const bool pq = pass[qi] && static_cast<uint32_t>(key[qi] >> 32) > thr[q];
+              seg_n[qi] = 0u;
+              seg_ptr[qi] = pools + (2 * qp + qi) * stride + p.cap + (a * 4 + quad) * seg_cap;
+            }
+          }
+          if (ok && (!half_parts || (quad >> 1) == ph)) {
+#pragma unroll
+            for (int qi = 0; qi < 2; ++qi) {
+              const bool pq = s < nvis[qi] && ord[qi] > thr_r[qi];
               const uint32_t bal = __ballot_sync(0xFFFFFFFFu, pq);
-              if (bal) {
-                uint32_t base = 0;
-                if (lane == 0) base = atomicAdd(&cnt[q], static_cast<uint32_t>(__popc(bal)));
-                base = __shfl_sync(0xFFFFFFFFu, base, 0);
-                if (pq) pool[q * p.pool_cap + base + __popc(bal & ((1u << lane) - 1u))] = key[qi];
-              }
+              if (pq)
+                seg_ptr[qi][seg_n[qi] + __popc(bal & ((1u << lane) - 1u))] =
+                    (static_cast<uint64_t>(ord[qi]) << 32) | low;
+              seg_n[qi] += __popc(bal);
             }
           }
-          const bool part_end = half_parts || ((j + 1) % part_tiles == 0) || (j == U.n_kt - 1);
-          if (part_end) {
-            epi_sync();
-            if (ew < QT && static_cast<int>(cnt[ew]) > k) {
-              thr[ew] = pool_shrink(pool + ew * p.pool_cap, cnt[ew], k, hist + ew * HIST_BINS, lane);
-              __syncwarp();
-              if (lane == 0) cnt[ew] = k;
+          const bool ends = half_parts || ((j + 1) % part_tiles == 0) || (j == U.n_kt - 1);
+          if (ends) {
+            __syncwarp();
+            if (lane == 0) {
+              C->seg_cnt[a][2 * qp][quad] = seg_n[0];
+              C->seg_cnt[a][2 * qp + 1][quad] = seg_n[1];
+              mbar_arrive(&C->seg_done[a][qp]);  // release: this warp's appends are visible
             }
-            epi_sync();
+            ++gp;
           }
         }
       }
-      // finalize: sort the <= k survivors of each query and store them
-      if (ew < QT) {
-        const int t = U.t0 + ew;
-        if (t < p.S) {
-          uint64_t* pl = pool + ew * p.pool_cap;
-          const int n = static_cast<int>(cnt[ew]);
-          int np = 32;
-          while (np < n) np <<= 1;
-          for (int x = n + lane; x < np; x += 32) pl[x] = 0ull;
-          __syncwarp();
-          warp_sort_desc(pl, np, lane);
-          const size_t ob = (static_cast<size_t>(U.b) * p.S + t) * static_cast<size_t>(k);
-          for (int x = lane; x < k; x += 32) {
-            int32_t id = -1;
-            float sc = -__int_as_float(0x7f800000);
-            if (x < n) {
-              const uint64_t key = pl[x];
-              id = static_cast<int32_t>(~static_cast<uint32_t>(key));
-              sc = ord_f32(static_cast<uint32_t>(key >> 32));
-            }
-            p.out_idx[ob + x] = id;
-            if (p.out_score) p.out_score[ob + x] = sc;
-          }
-        }
-      }
-      epi_sync();
     }
   }
 
@@ -613,20 +599,29 @@ bool stream_smem_plan(int k, int key_tile, int fp8, int* n_stages, int* pool_cap
   const int opb = fp8 ? 1 : 2;
   int np2 = 32;
   while (np2 < k) np2 <<= 1;
-  const int cap = std::max(k + key_tile, np2);
+  const int seg_cap = seg_capacity(key_tile);
+  const int room = key_tile;  // one partition's appends
+  // the main region takes a whole partition on top of k survivors, holds the
+  // padded final sort, and, when shared memory allows, up to k more so
+  // compaction stays rare
+  const int cap_min = std::max(k + room, np2);
+  const int cap_want = std::max(cap_min, 2 * k + room);
   const size_t q_bytes = static_cast<size_t>(NCOLS) * DIM * opb;
   const size_t kc_bytes = static_cast<size_t>(KT) * DIM * opb;
-  const size_t fixed = q_bytes + static_cast<size_t>(QT) * cap * 8 + QT * HEADS * 4 +
-                       QT * HIST_BINS * 4 + 256 + 1024 /* alignment slack */;
   const size_t limit = 227 * 1024;
+  const size_t areas = static_cast<size_t>(QT) * N_AREAS * 4 * seg_cap * 8;
   for (int ns = 4; ns >= 2; --ns) {
-    const size_t tot = fixed + ns * kc_bytes;
-    if (tot <= limit) {
-      *n_stages = ns;
-      *pool_cap = cap;
-      *bytes = tot;
-      return true;
-    }
+    const size_t fixed = q_bytes + ns * kc_bytes + areas + QT * HIST_BINS * 4 + CTRL_BYTES +
+                         1024 /* alignment slack */;
+    if (fixed >= limit) continue;
+    const int cap_max = static_cast<int>((limit - fixed) / (QT * 8));
+    if (cap_max < cap_min) continue;
+    if (ns == 4 && cap_max < cap_want) continue;  // a larger pool beats a fourth stage
+    const int cap = std::min(cap_max, cap_want);
+    *n_stages = ns;
+    *pool_cap = cap;
+    *bytes = fixed + static_cast<size_t>(QT) * cap * 8;
+    return true;
   }
   return false;
 }
@@ -636,9 +631,9 @@ si_status launch_stream_topk(const void* q, const void* kc, const float* w, int 
                              cudaStream_t stream, const StreamConfig& cfg) {
   (void)H;
   (void)D;
-  int n_stages = 0, pool_cap = 0;
+  int n_stages = 0, cap = 0;
   size_t smem = 0;
-  if (!stream_smem_plan(k, cfg.key_tile, cfg.fp8, &n_stages, &pool_cap, &smem))
+  if (!stream_smem_plan(k, cfg.key_tile, cfg.fp8, &n_stages, &cap, &smem))
     return fail(SI_ERR_UNSUPPORTED, "k=%d with key_tile=%d does not fit in shared memory", k, cfg.key_tile);
   const int opb = cfg.fp8 ? 1 : 2;
   const CUtensorMapDataType dt = cfg.fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -677,7 +672,7 @@ si_status launch_stream_topk(const void* q, const void* kc, const float* w, int 
   p.m = m;
   p.k = k;
   p.key_tile = cfg.key_tile;
-  p.pool_cap = pool_cap;
+  p.cap = cap;
   p.n_stages = n_stages;
   p.wait_limit_ns = cfg.wait_limit_ns;
   p.test_withhold = cfg.test_withhold;

@@ -8,7 +8,12 @@ Acceptance rules (the indexer top-k's contract):
     oracle's j-th score (absolute floor 1e-6 * the row's largest score), every
     index that is in one set but not the other has an oracle score within a
     1e-3 relative tie window of the oracle's k-th score, and set-overlap
-    recall |G & O| / |O| has mean >= 0.9999 and min >= 0.998;
+    recall |G & O| / |O| has mean >= 0.9999 and min >= 0.998, where a
+    returned index whose oracle score lies within ROUND_WIN (1e-5) relative of
+    the oracle's k-th score counts as a hit: two fp32 evaluations of one
+    score differ by ~1e-7 relative, so such a key ties the k-th one within
+    rounding and which of them is kept is arbitrary.  Raw recall (no such
+    allowance) is returned too.
   * always: valid entries = min(k, visible keys), -1 / -inf padding after
     them, distinct indices, every index causally visible, scores sorted
     descending.
@@ -24,6 +29,7 @@ import oracle
 import synth
 
 REL = 1e-3
+ROUND_WIN = 1e-5
 ABS_FLOOR = 1e-6
 RECALL_MEAN = 0.9999
 RECALL_MIN = 0.998
@@ -67,6 +73,19 @@ def oracle_rows(wl_name: str, rows: np.ndarray, k: int, fmt: str = "bf16", overr
     return idx, sc, sc64
 
 
+def report(name: str, key: str, value) -> None:
+    """Append a result to $SI_REPORT_DIR/<name>.json when that variable is set."""
+    d = os.environ.get("SI_REPORT_DIR")
+    if not d:
+        return
+    import json
+    os.makedirs(d, exist_ok=True)
+    path = os.path.join(d, f"{name}.json")
+    data = json.load(open(path)) if os.path.exists(path) else {}
+    data[key] = value
+    json.dump(data, open(path, "w"), indent=1, sort_keys=True)
+
+
 def check_structure(idx: np.ndarray, score: np.ndarray, rows: np.ndarray, S: int, T: int, m: int):
     """Padding, distinctness, causal visibility and order of GPU rows."""
     k = idx.shape[1]
@@ -88,10 +107,13 @@ def compare_exact(gi, gs, oi, osc, rows):
                            f"oracle {oi[bad[0], :8]}")
 
 
-def compare_tolerant(gi, gs, oi, osc64, rows, score_row_fn):
-    """Returns (mean recall, min recall).  score_row_fn(row) -> oracle scores
-    of all keys of that row (double), used only for rows with a mismatch."""
-    recalls = []
+def compare_tolerant(gi, gs, oi, osc64, rows, score_row_fn, details=None):
+    """Returns (mean recall, min recall) with rounding ties counted as hits.
+    score_row_fn(row) -> oracle scores of all keys of that row (double), used
+    only for rows with a mismatch.  `details` (a dict) receives raw recall and
+    the largest relative gap of a mismatched key to the k-th score."""
+    recalls, raw = [], []
+    max_gap = 0.0
     for r in range(len(rows)):
         nv = int((oi[r] >= 0).sum())
         if nv == 0:
@@ -103,12 +125,20 @@ def compare_tolerant(gi, gs, oi, osc64, rows, score_row_fn):
         err = np.abs(g - o)
         assert np.all(err <= REL * np.abs(o) + floor), (rows[r], float(err.max()))
         G, O = set(gi[r, :nv].tolist()), set(oi[r, :nv].tolist())
-        recalls.append(len(G & O) / nv)
+        hits = len(G & O)
+        raw.append(hits / nv)
         if G != O:
             allsc = score_row_fn(int(rows[r]))
             kth = o[-1]
             win = REL * abs(kth) + floor
             for x in G ^ O:
-                assert abs(allsc[x] - kth) <= win, (rows[r], x, allsc[x], kth)
+                gap = abs(allsc[x] - kth)
+                assert gap <= win, (rows[r], x, allsc[x], kth)
+                max_gap = max(max_gap, gap / max(abs(kth), 1e-30))
+            hits += sum(1 for x in G - O if abs(allsc[x] - kth) <= ROUND_WIN * abs(kth) + floor)
+        recalls.append(min(1.0, hits / nv))
     rec = np.asarray(recalls) if recalls else np.ones(1)
+    rr = np.asarray(raw) if raw else np.ones(1)
+    if details is not None:
+        details.update(raw_mean=float(rr.mean()), raw_min=float(rr.min()), max_gap_rel=max_gap)
     return float(rec.mean()), float(rec.min())
