@@ -103,6 +103,31 @@ SI_API si_status si_indexer_materialize(const void* q, const void* kc, const flo
                                  int T, int H_I, int D, int m, int k, int32_t* out_idx,
                                  float* out_score, void* stream, const si_options* opt);
 
+/*
+ * Allocation-free variant of si_indexer_materialize, for callers that cannot
+ * allocate device memory at call time (an application that has given nearly
+ * all GPU memory to its own pool, a plugin step that must not allocate, a
+ * latency-critical loop where cudaMalloc/cudaFree would synchronise).  It has
+ * no counterpart on the pages: it runs the same materialize kernels with
+ * their scratch in a fixed device array of SI_NOALLOC_SCRATCH_BYTES that the
+ * library holds on every GPU that loads it, until the process exits.
+ *   Same arguments, layouts, ownership and results as
+ *   si_indexer_materialize (bf16 q, kc; fp32 w; device pointers).
+ *   Returns SI_ERR_UNSUPPORTED, touching nothing, when the scratch need
+ *   4*B*S*T*(H_I+1) + 256 bytes exceeds SI_NOALLOC_SCRATCH_BYTES, or T >
+ *   16384.  Calls no cudaMalloc / cudaFree and nothing that allocates.
+ *   The first call on a device looks up the array's device address (once per
+ *   device, with that device current); make that first call before any
+ *   stream capture.
+ *   All calls on a device share the array, which keeps the last call's
+ *   contents (every word is overwritten before it is read); calls whose
+ *   work overlaps on the same device race on it and must be serialised.
+ */
+#define SI_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+SI_API si_status si_indexer_materialize_noalloc(const void* q, const void* kc, const float* w,
+                                                int B, int S, int T, int H_I, int D, int m, int k,
+                                                int32_t* out_idx, float* out_score, void* stream);
+
 /* Scratch bytes a call with these arguments needs (0 if none).  materialize
  * selects the materialize path's need. */
 SI_API size_t si_indexer_workspace_size(int B, int S, int T, int H_I, int D, int m, int k, int materialize,

@@ -45,6 +45,9 @@ _lib.si_indexer_topk_ex.restype = _i
 _lib.si_indexer_topk_ex.argtypes = _ARGS + [ctypes.POINTER(Options)]
 _lib.si_indexer_materialize.restype = _i
 _lib.si_indexer_materialize.argtypes = _ARGS + [ctypes.POINTER(Options)]
+_lib.si_indexer_materialize_noalloc.restype = _i
+_lib.si_indexer_materialize_noalloc.argtypes = _ARGS
+NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024  # SI_NOALLOC_SCRATCH_BYTES
 _lib.si_indexer_workspace_size.restype = _sz
 _lib.si_indexer_workspace_size.argtypes = [_i] * 8 + [ctypes.POINTER(Options)]
 _lib.si_device_status.restype = _i
@@ -151,6 +154,22 @@ def indexer_materialize(q, kc, w, m: int, k: int, *, out_idx=None, out_score=Non
                                      out_score.data_ptr() if out_score is not None else None,
                                      _stream_ptr(stream), ctypes.byref(o))
     _check(st, "si_indexer_materialize")
+    return out_idx, out_score
+
+
+def indexer_materialize_noalloc(q, kc, w, m: int, k: int, *, out_idx=None, out_score=None,
+                                with_score: bool = True, stream=None):
+    """Materialize path without device allocation (``si_indexer_materialize_noalloc``):
+    its scratch is the library's fixed device array of NOALLOC_SCRATCH_BYTES.
+    For callers that may not allocate device memory during the call; pass
+    preallocated outputs to keep the call itself allocation-free."""
+    B, S, T, H, D = _shapes(q, kc, w)
+    out_idx, out_score = _outputs(B, S, k, q.device, out_idx, out_score, with_score)
+    st = _lib.si_indexer_materialize_noalloc(q.data_ptr(), kc.data_ptr(), w.data_ptr(), B, S, T, H, D, m,
+                                             k, out_idx.data_ptr(),
+                                             out_score.data_ptr() if out_score is not None else None,
+                                             _stream_ptr(stream))
+    _check(st, "si_indexer_materialize_noalloc")
     return out_idx, out_score
 
 

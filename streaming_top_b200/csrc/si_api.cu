@@ -86,8 +86,6 @@ si_status encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void
   return SI_OK;
 }
 
-namespace {
-
 si_status check_common(const void* q, const void* kc, const float* w, int B, int S, int T, int H,
                        int D, int m, int k, const int32_t* out_idx, const float* out_score) {
   if (!q || !kc || !w || !out_idx)
@@ -101,7 +99,6 @@ si_status check_common(const void* q, const void* kc, const float* w, int B, int
   return SI_OK;
 }
 
-}  // namespace
 }  // namespace si
 
 using namespace si;

@@ -15,6 +15,10 @@ namespace si {
 si_status fail(si_status st, const char* fmt, ...);
 // Converts a CUDA runtime error into SI_ERR_CUDA with context.
 si_status cuda_fail(cudaError_t e, const char* what);
+// Host-side checks shared by every entry point: non-null pointers, sizes
+// >= 1, 16-byte aligned inputs, 4-byte aligned outputs.
+si_status check_common(const void* q, const void* kc, const float* w, int B, int S, int T, int H,
+                       int D, int m, int k, const int32_t* out_idx, const float* out_score);
 
 // Device-resident error record of this library on the current device:
 // int[4] = {code, where, detail, spare}.  code 0 = none, SI_ERR_TIMEOUT =
