@@ -50,7 +50,7 @@ def load_peaks() -> dict:
 
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
-    for f in ("si_stream.cu", "si_ptx.cuh"):
+    for f in ("si_stream.cu", "si_topk.cuh", "si_ptx.cuh"):
         h.update(open(os.path.join(ROOT, "streaming_top_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -126,6 +126,25 @@ def config_dict(wl, n_gpus: int) -> dict:
 
 
 # ------------------------------------------------------------------ CPU oracle
+def rank_seed(wl, rank: int) -> int:
+    """Each rank runs its own independent sequences of the same shape."""
+    return wl.seed + 1000 * rank
+
+
+def max_over_ranks(x: float, device) -> float:
+    """The slowest rank's figure (all ranks must call this, in the same order)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(world: int, pairs_per_rank: int, ms_step: float) -> float:
+    """Whole-job throughput: every rank's pairs over the slowest rank's time."""
+    return world * pairs_per_rank / (ms_step * 1e-3)
+
+
 def oracle_sample(wl, inp, rows) -> tuple[float, int]:
     import oracle
     t0 = time.perf_counter()
@@ -186,7 +205,7 @@ def run_ours(args, wl):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
 
-    seed = wl.seed + 1000 * rank  # each rank: its own sequence of the same shape
+    seed = rank_seed(wl, rank)
     inp = synth.make_inputs(wl, seed=seed)
     q = torch.from_numpy(inp["q"].view(np.int16)).view(torch.bfloat16).to(dev)
     kc = torch.from_numpy(inp["kc"].view(np.int16)).view(torch.bfloat16).to(dev)
@@ -234,9 +253,7 @@ def run_ours(args, wl):
     ms_step = sum(ms) / len(ms)
     peak_mem = torch.cuda.max_memory_allocated(dev)
     if world > 1:
-        t = torch.tensor([ms_step], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step = float(t.item())
+        ms_step = max_over_ranks(ms_step, dev)
 
     # end to end through the host-buffer API: H2D inputs, kernel, D2H results
     hq = torch.from_numpy(inp["q"].view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -257,9 +274,7 @@ def run_ours(args, wl):
     torch.cuda.synchronize(dev)
     e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev) / args.steps
     if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(e2e_ms, dev)
     h2d = hq.numel() * 2 + hk.numel() * 2 + hw.numel() * 4
     d2h = out_idx.numel() * 4 + out_score.numel() * 4
     del bufs
@@ -273,7 +288,7 @@ def run_ours(args, wl):
     P = wl.visible_pairs()
     flop_pair = 2 * wl.H * wl.D
     peaks = load_peaks()
-    value = world * P / (ms_step * 1e-3)
+    value = job_value(world, P, ms_step)
     tflops = P * flop_pair / (ms_step * 1e-3) / 1e12
     alg_bytes = q.numel() * 2 + kc.numel() * 2 + w.numel() * 4 + out_idx.numel() * 4 + out_score.numel() * 4
     traffic = ncu_traffic(wl.name)
@@ -310,7 +325,7 @@ def run_ours(args, wl):
                      "peak_source": f"{peaks['source']} bf16 dense matmul, burst",
                      "traffic": traffic, "algorithmic_bytes": alg_bytes},
         "cpu_baseline": cpu,
-        "e2e": {"value": world * P / (e2e_ms * 1e-3), "unit": "pairs/s", "h2d_bytes_per_step": h2d,
+        "e2e": {"value": job_value(world, P, e2e_ms), "unit": "pairs/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": args.steps,
         "clocks": clocks,
