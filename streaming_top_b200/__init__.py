@@ -109,13 +109,20 @@ def _outputs(B, S, k, device, out_idx, out_score, with_score):
     return out_idx, out_score
 
 
-def _options(q, q_scale, kc_scale, query_chunk, key_tile, workspace=None):
+def _options(q, kc, q_scale, kc_scale, query_chunk, key_tile, workspace=None):
     o = Options()
+    if kc.element_size() != q.element_size():
+        raise ValueError(f"q ({q.dtype}) and kc ({kc.dtype}) must have the same element type")
     if q.dtype == torch.bfloat16:
         o.dtype = SI_DTYPE_BF16
     elif q.dtype in (torch.uint8, torch.float8_e4m3fn):
         if q_scale is None or kc_scale is None:
             raise ValueError("fp8 inputs need q_scale and kc_scale")
+        B, S, H, _ = q.shape
+        for name, t, shape in (("q_scale", q_scale, (B, S, H)), ("kc_scale", kc_scale, (B, kc.shape[1]))):
+            if (t.dtype != torch.float32 or tuple(t.shape) != shape or not t.is_cuda
+                    or not t.is_contiguous()):
+                raise ValueError(f"{name} must be a contiguous float32 CUDA tensor of shape {shape}")
         o.dtype = SI_DTYPE_FP8_E4M3
         o.q_scale = q_scale.data_ptr()
         o.kc_scale = kc_scale.data_ptr()
@@ -135,7 +142,7 @@ def indexer_topk(q, kc, w, m: int, k: int, *, q_scale=None, kc_scale=None, query
     """Streaming indexer top-k (``si_indexer_topk_ex``).  Returns (idx, score)."""
     B, S, T, H, D = _shapes(q, kc, w)
     out_idx, out_score = _outputs(B, S, k, q.device, out_idx, out_score, with_score)
-    o = _options(q, q_scale, kc_scale, query_chunk, key_tile)
+    o = _options(q, kc, q_scale, kc_scale, query_chunk, key_tile)
     st = _lib.si_indexer_topk_ex(q.data_ptr(), kc.data_ptr(), w.data_ptr(), B, S, T, H, D, m, k,
                                  out_idx.data_ptr(), out_score.data_ptr() if out_score is not None else None,
                                  _stream_ptr(stream), ctypes.byref(o))
@@ -148,7 +155,7 @@ def indexer_materialize(q, kc, w, m: int, k: int, *, out_idx=None, out_score=Non
     """Materialize-path ground truth (``si_indexer_materialize``)."""
     B, S, T, H, D = _shapes(q, kc, w)
     out_idx, out_score = _outputs(B, S, k, q.device, out_idx, out_score, with_score)
-    o = _options(q, None, None, 0, 0, workspace)
+    o = _options(q, kc, None, None, 0, 0, workspace)
     st = _lib.si_indexer_materialize(q.data_ptr(), kc.data_ptr(), w.data_ptr(), B, S, T, H, D, m, k,
                                      out_idx.data_ptr(),
                                      out_score.data_ptr() if out_score is not None else None,

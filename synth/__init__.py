@@ -52,6 +52,10 @@ def lib():
         L.synth_matrix.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
                                    ctypes.c_uint64, ctypes.c_uint32, ctypes.c_int, ctypes.c_double,
                                    ctypes.c_int, ctypes.c_int]
+        L.synth_matrix_range.restype = ctypes.c_int
+        L.synth_matrix_range.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                                         ctypes.c_int, ctypes.c_uint64, ctypes.c_uint32, ctypes.c_int,
+                                         ctypes.c_double, ctypes.c_int, ctypes.c_int]
         L.synth_keys_planted.restype = ctypes.c_int
         L.synth_keys_planted.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
                                          ctypes.c_int, ctypes.c_uint64, ctypes.c_uint32, ctypes.c_double,
@@ -90,6 +94,30 @@ def matrix(rows: int, D: int, seed: int, tensor_id: int, kind: str = "gauss", si
     o = out if out is not None else np.empty((rows, D), dtype=np.uint8)
     s = scale_out if scale_out is not None else np.empty((rows,), dtype=np.float32)
     rc = lib().synth_matrix(_ptr(o), _ptr(s), rows, D, seed, tensor_id, k, sigma, 1, _threads())
+    assert rc == 0
+    return o, s
+
+
+def matrix_range(row0: int, rows: int, D: int, seed: int, tensor_id: int, kind: str = "gauss",
+                 sigma: float = 1.0, fmt: str = "bf16", out: np.ndarray | None = None,
+                 scale_out: np.ndarray | None = None):
+    """Rows [row0, row0+rows) of `matrix(...)` with the same arguments: the
+    same values, generated alone (out / scale_out receive them from their
+    first element on)."""
+    k = {"gauss": 0, "int": 1}[kind]
+    if fmt == "bf16":
+        o = out if out is not None else np.empty((rows, D), dtype=np.uint16)
+        assert o.dtype == np.uint16 and o.flags.c_contiguous and o.size >= rows * D
+        rc = lib().synth_matrix_range(_ptr(o), None, row0, rows, D, seed, tensor_id, k, sigma, 0,
+                                      _threads())
+        assert rc == 0
+        return o
+    o = out if out is not None else np.empty((rows, D), dtype=np.uint8)
+    s = scale_out if scale_out is not None else np.empty((rows,), dtype=np.float32)
+    assert o.dtype == np.uint8 and o.flags.c_contiguous and o.size >= rows * D
+    assert s.dtype == np.float32 and s.flags.c_contiguous and s.size >= rows
+    rc = lib().synth_matrix_range(_ptr(o), _ptr(s), row0, rows, D, seed, tensor_id, k, sigma, 1,
+                                  _threads())
     assert rc == 0
     return o, s
 
@@ -197,13 +225,15 @@ PLANTED_BOOST = 2.0
 
 
 def make_inputs(wl: Workload, fmt: str = "bf16", S: int | None = None, B: int | None = None,
-                seed: int | None = None):
+                seed: int | None = None, skip_q: bool = False):
     """Generate (q, kc, w[, q_scale, kc_scale]) host arrays for a workload.
 
     q: [B, S, H, D] (bf16 bits uint16, or e4m3 uint8 + q_scale [B, S, H])
     kc: [B, T, D]   (bf16 bits, or e4m3 + kc_scale [B, T])
     w: [B, S, H] float32
     `S`, `B` and `seed` override the workload's (for reduced-size cases).
+    `skip_q` leaves q (and q_scale) out, for callers that make it piecewise
+    with q_rows().
     """
     S = wl.S if S is None else S
     B = wl.B if B is None else B
@@ -214,7 +244,9 @@ def make_inputs(wl: Workload, fmt: str = "bf16", S: int | None = None, B: int | 
     kind = "int" if wl.kind == "int" else "gauss"
     qsig = 1.0 if kind == "int" else sig
     res = {}
-    if fmt == "bf16":
+    if skip_q:
+        q = None
+    elif fmt == "bf16":
         q = matrix(B * S * H, D, seed, TENSOR_Q, kind, qsig, "bf16").reshape(B, S, H, D)
     else:
         q8, qs = matrix(B * S * H, D, seed, TENSOR_Q, kind, qsig, "e4m3")
@@ -233,5 +265,49 @@ def make_inputs(wl: Workload, fmt: str = "bf16", S: int | None = None, B: int | 
         w = weights(B * S * H, seed, TENSOR_W, "pow2").reshape(B, S, H)
     else:
         w = weights(B * S * H, seed, TENSOR_W, "uniform", 1.0 / np.sqrt(H)).reshape(B, S, H)
-    res.update(q=q, kc=kc, w=w)
+    res.update(kc=kc, w=w)
+    if q is not None:
+        res["q"] = q
     return res
+
+
+def _q_kind(wl: Workload):
+    kind = "int" if wl.kind == "int" else "gauss"
+    return kind, (1.0 if kind == "int" else 1.0 / np.sqrt(wl.D))
+
+
+def q_rows(wl: Workload, b: int, t0: int, n: int, fmt: str = "bf16", seed: int | None = None,
+           S: int | None = None, out: np.ndarray | None = None, scale_out: np.ndarray | None = None):
+    """q[b, t0:t0+n] of make_inputs(wl, fmt, S, seed=seed), generated alone:
+    [n, H, D] bf16 bits, or (e4m3 codes, q_scale [n, H])."""
+    S = wl.S if S is None else S
+    seed = wl.seed if seed is None else seed
+    kind, sig = _q_kind(wl)
+    row0 = (b * S + t0) * wl.H
+    res = matrix_range(row0, n * wl.H, wl.D, seed, TENSOR_Q, kind, sig, fmt, out=out, scale_out=scale_out)
+    if fmt == "bf16":
+        return res.reshape(n, wl.H, wl.D)
+    return res[0].reshape(n, wl.H, wl.D), res[1].reshape(n, wl.H)
+
+
+def make_inputs_rows(wl: Workload, rows, fmt: str = "bf16", seed: int | None = None):
+    """make_inputs(wl, fmt, seed=seed) with q (and q_scale) generated only at
+    the given flat query rows b*S+t; kc and w are complete.  The other q rows
+    are left unwritten in a lazily allocated array, so a few rows of a
+    million-token sequence cost a few MiB of host memory."""
+    seed = wl.seed if seed is None else seed
+    B, S, T, H, D = wl.B, wl.S, wl.T, wl.H, wl.D
+    full = make_inputs(wl, fmt=fmt, S=S, B=B, seed=seed, skip_q=True)
+    qdt = np.uint16 if fmt == "bf16" else np.uint8
+    q = np.empty((B, S, H, D), dtype=qdt)
+    qs = np.empty((B, S, H), dtype=np.float32) if fmt != "bf16" else None
+    for r in np.asarray(rows, dtype=np.int64):
+        b, t = divmod(int(r), S)
+        if fmt == "bf16":
+            q_rows(wl, b, t, 1, fmt, seed, out=q[b, t])
+        else:
+            q_rows(wl, b, t, 1, fmt, seed, out=q[b, t], scale_out=qs[b, t])
+    full["q"] = q
+    if qs is not None:
+        full["q_scale"] = qs
+    return full

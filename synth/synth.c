@@ -119,6 +119,7 @@ enum { FMT_BF16 = 0, FMT_E4M3 = 1 };
 typedef struct {
   void* out; float* scale; int D; int kind; int fmt;
   uint64_t key; double sigma;
+  int64_t row0; /* global index of out's first row (element counter base) */
   /* planted boost (kc only) */
   const uint8_t* boosted; const float* dir; int T; double boost;
 } rows_ctx;
@@ -145,7 +146,7 @@ static void rows_work(void* p, int64_t r0, int64_t r1) {
     const float* dir = NULL;
     if (c->boosted && c->boosted[r]) dir = c->dir + (r / c->T) * c->D;
     for (int d = 0; d < c->D; ++d) {
-      uint64_t i = (uint64_t)r * c->D + d;
+      uint64_t i = (uint64_t)(c->row0 + r) * c->D + d;
       double v;
       if (c->kind == KIND_GAUSS) v = synth_normal(c->key, i) * c->sigma;
       else v = (double)(u_below(synth_draw(c->key, i), 7) - 3);
@@ -168,6 +169,22 @@ int synth_matrix(void* out, float* scale, int64_t rows, int D, uint64_t seed,
   memset(&c, 0, sizeof c);
   c.out = out; c.scale = scale; c.D = D; c.kind = kind; c.fmt = fmt;
   c.key = synth_stream_key(seed, tensor_id); c.sigma = sigma;
+  parallel_rows(rows_work, &c, rows, nthreads);
+  return 0;
+}
+
+/*
+ * Rows [row0, row0 + rows) of the matrix synth_matrix would make, written to
+ * out (and scale) starting at their first element: the same values, for
+ * callers that fill a large tensor piecewise or need a few rows only.
+ */
+int synth_matrix_range(void* out, float* scale, int64_t row0, int64_t rows, int D, uint64_t seed,
+                       uint32_t tensor_id, int kind, double sigma, int fmt, int nthreads) {
+  if (D <= 0 || D > 1024 || rows < 0 || row0 < 0 || (fmt == FMT_E4M3 && !scale)) return -1;
+  rows_ctx c;
+  memset(&c, 0, sizeof c);
+  c.out = out; c.scale = scale; c.D = D; c.kind = kind; c.fmt = fmt;
+  c.key = synth_stream_key(seed, tensor_id); c.sigma = sigma; c.row0 = row0;
   parallel_rows(rows_work, &c, rows, nthreads);
   return 0;
 }

@@ -36,21 +36,25 @@ RECALL_MIN = 0.998
 
 
 def _worker(args):
-    wl_name, overrides, fmt, k, rows = args
+    wl_name, overrides, fmt, k, rows, sparse = args
     wl = synth.WORKLOADS[wl_name]
-    inp = synth.make_inputs(wl, fmt=fmt, **overrides)
+    if sparse:  # only this worker's q rows (a million-token q is 16 GiB)
+        inp = synth.make_inputs_rows(wl, rows, fmt=fmt, **overrides)
+    else:
+        inp = synth.make_inputs(wl, fmt=fmt, **overrides)
     idx, sc, sc64 = oracle.topk(inp["q"], inp["kc"], inp["w"], wl.m, k, rows=rows,
                                 q_scale=inp.get("q_scale"), kc_scale=inp.get("kc_scale"))
     return idx, sc, sc64
 
 
 def oracle_rows(wl_name: str, rows: np.ndarray, k: int, fmt: str = "bf16", overrides=None,
-                procs: int | None = None, inputs=None):
+                procs: int | None = None, inputs=None, sparse: bool = False):
     """Oracle (idx, score, score64) for flat rows of a named workload.
 
     With `inputs` (the exact host arrays given to the GPU) it runs in this
     process; otherwise the rows are split over a spawn pool whose workers
-    regenerate the same seeded inputs."""
+    regenerate the same seeded inputs (with `sparse`, only the q rows they
+    need)."""
     rows = np.asarray(rows, dtype=np.int64)
     wl = synth.WORKLOADS[wl_name]
     if inputs is not None:
@@ -61,7 +65,7 @@ def oracle_rows(wl_name: str, rows: np.ndarray, k: int, fmt: str = "bf16", overr
     parts = [rows[i::procs] for i in range(procs) if len(rows[i::procs])]
     ctx = mp.get_context("spawn")
     with ctx.Pool(len(parts)) as pool:
-        res = pool.map(_worker, [(wl_name, overrides or {}, fmt, k, p) for p in parts])
+        res = pool.map(_worker, [(wl_name, overrides or {}, fmt, k, p, sparse) for p in parts])
     n = len(rows)
     idx = np.empty((n, k), np.int32)
     sc = np.empty((n, k), np.float32)

@@ -1,5 +1,6 @@
 """The seeded input generator (no GPU)."""
 import numpy as np
+import pytest
 import torch
 
 import synth
@@ -100,3 +101,24 @@ def test_visible_pairs_closed_form():
     wl = synth.WORKLOADS["v4flash"]
     assert wl.visible_pairs() == 536854528
     assert synth.WORKLOADS["million"].visible_pairs() == 137438691328
+
+
+@pytest.mark.parametrize("name,fmt", [("tiny", "bf16"), ("tiny", "e4m3"), ("integer", "bf16"),
+                                      ("integer", "e4m3")])
+def test_rows_generated_alone_equal_the_full_tensor(name, fmt):
+    """q_rows / make_inputs_rows give exactly the rows of make_inputs."""
+    wl = synth.WORKLOADS[name]
+    full = synth.make_inputs(wl, fmt=fmt)
+    rows = np.array([0, 5, 777, wl.S - 1])
+    part = synth.make_inputs_rows(wl, rows, fmt=fmt)
+    for r in rows:
+        assert np.array_equal(full["q"][0, r], part["q"][0, r])
+        if fmt != "bf16":
+            assert np.array_equal(full["q_scale"][0, r], part["q_scale"][0, r])
+    assert np.array_equal(full["kc"], part["kc"]) and np.array_equal(full["w"], part["w"])
+    blk = synth.q_rows(wl, 0, 100, 37, fmt)
+    if fmt == "bf16":
+        assert np.array_equal(blk, full["q"][0, 100:137])
+    else:
+        assert np.array_equal(blk[0], full["q"][0, 100:137])
+        assert np.array_equal(blk[1], full["q_scale"][0, 100:137])
