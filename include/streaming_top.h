@@ -69,6 +69,9 @@ typedef struct si_options {
                             of 128 up to 1024; 0 = 512 */
   void* workspace;       /* optional caller-owned device scratch, >= si_indexer_workspace_size() */
   size_t workspace_bytes;
+  int unsorted;          /* streaming path only: 1 = leave each row's k results in an unspecified
+                            order (valid entries first, then the -1 / -inf padding) and skip the
+                            row sort; 0 (default) = sorted by score descending, index ascending */
 } si_options;
 
 /*
@@ -89,6 +92,17 @@ SI_API si_status si_indexer_topk(const void* q, const void* kc, const float* w, 
 SI_API si_status si_indexer_topk_ex(const void* q, const void* kc, const float* w, int B, int S, int T,
                              int H_I, int D, int m, int k, int32_t* out_idx, float* out_score,
                              void* stream, const si_options* opt);
+
+/*
+ * Sorts every row of a top-k result in place by (score descending, index
+ * ascending): idx [rows, k] int32, score [rows, k] fp32, device memory, one
+ * row per query.  Entries with index -1 and score -inf (padding) end up last.
+ * This is the step si_indexer_topk runs after the streaming kernel when
+ * out_score is given; callers that ran si_indexer_topk_ex with `unsorted`
+ * can run it later.  Scores must not be NaN.  rows >= 0, 1 <= k <= 2048;
+ * idx and score 4-byte aligned.  Asynchronous on `stream`.
+ */
+SI_API si_status si_sort_topk_rows(int32_t* idx, float* score, int64_t rows, int k, void* stream);
 
 /*
  * Materialize path (in-library ground truth for small S, the method the

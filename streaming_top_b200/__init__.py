@@ -35,7 +35,7 @@ _vp, _i, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
 
 class Options(ctypes.Structure):
     _fields_ = [("dtype", _i), ("q_scale", _vp), ("kc_scale", _vp), ("query_chunk", _i),
-                ("key_tile", _i), ("workspace", _vp), ("workspace_bytes", _sz)]
+                ("key_tile", _i), ("workspace", _vp), ("workspace_bytes", _sz), ("unsorted", _i)]
 
 
 _ARGS = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp]
@@ -43,6 +43,8 @@ _lib.si_indexer_topk.restype = _i
 _lib.si_indexer_topk.argtypes = _ARGS
 _lib.si_indexer_topk_ex.restype = _i
 _lib.si_indexer_topk_ex.argtypes = _ARGS + [ctypes.POINTER(Options)]
+_lib.si_sort_topk_rows.restype = _i
+_lib.si_sort_topk_rows.argtypes = [_vp, _vp, ctypes.c_int64, _i, _vp]
 _lib.si_indexer_materialize.restype = _i
 _lib.si_indexer_materialize.argtypes = _ARGS + [ctypes.POINTER(Options)]
 _lib.si_indexer_materialize_noalloc.restype = _i
@@ -138,16 +140,34 @@ def _options(q, kc, q_scale, kc_scale, query_chunk, key_tile, workspace=None):
 
 def indexer_topk(q, kc, w, m: int, k: int, *, q_scale=None, kc_scale=None, query_chunk: int = 0,
                  key_tile: int = 0, out_idx=None, out_score=None, with_score: bool = True,
-                 stream=None):
-    """Streaming indexer top-k (``si_indexer_topk_ex``).  Returns (idx, score)."""
+                 unsorted: bool = False, stream=None):
+    """Streaming indexer top-k (``si_indexer_topk_ex``).  Returns (idx, score).
+    With unsorted=True each row's results come in an unspecified order (valid
+    entries first) and the row sort is skipped."""
     B, S, T, H, D = _shapes(q, kc, w)
     out_idx, out_score = _outputs(B, S, k, q.device, out_idx, out_score, with_score)
     o = _options(q, kc, q_scale, kc_scale, query_chunk, key_tile)
+    o.unsorted = int(bool(unsorted))
     st = _lib.si_indexer_topk_ex(q.data_ptr(), kc.data_ptr(), w.data_ptr(), B, S, T, H, D, m, k,
                                  out_idx.data_ptr(), out_score.data_ptr() if out_score is not None else None,
                                  _stream_ptr(stream), ctypes.byref(o))
     _check(st, "si_indexer_topk_ex")
     return out_idx, out_score
+
+
+def sort_topk_rows(idx, score, stream=None):
+    """Sort every row of (idx [..., k] int32, score [..., k] fp32) in place by
+    score descending, index ascending (``si_sort_topk_rows``)."""
+    if idx.shape != score.shape or idx.dtype != torch.int32 or score.dtype != torch.float32:
+        raise ValueError("idx int32 and score float32 of the same shape expected")
+    for name, t in (("idx", idx), ("score", score)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    k = idx.shape[-1]
+    rows = idx.numel() // k if k else 0
+    _check(_lib.si_sort_topk_rows(idx.data_ptr(), score.data_ptr(), rows, k, _stream_ptr(stream)),
+           "si_sort_topk_rows")
+    return idx, score
 
 
 def indexer_materialize(q, kc, w, m: int, k: int, *, out_idx=None, out_score=None,

@@ -135,8 +135,23 @@ si_status si_indexer_topk_ex(const void* q, const void* kc, const float* w, int 
   cfg.kc_scale = o.kc_scale;
   cfg.wait_limit_ns = kDefaultWaitLimitNs;
   cfg.test_withhold = 0;
-  return launch_stream_topk(q, kc, w, B, S, T, H_I, D, m, k, out_idx, out_score,
-                            static_cast<cudaStream_t>(stream), cfg);
+  cfg.unsorted = o.unsorted != 0;
+  st = launch_stream_topk(q, kc, w, B, S, T, H_I, D, m, k, out_idx, out_score,
+                          static_cast<cudaStream_t>(stream), cfg);
+  if (st != SI_OK || cfg.unsorted || !out_score) return st;
+  // the kernel left each row's k results in pool order: sort them now
+  return launch_row_sort(out_idx, out_score, static_cast<long long>(B) * S, k,
+                         static_cast<cudaStream_t>(stream));
+}
+
+si_status si_sort_topk_rows(int32_t* idx, float* score, int64_t rows, int k, void* stream) {
+  if (rows < 0) return fail(SI_ERR_INVALID_ARGUMENT, "rows must be >= 0 (got %lld)", static_cast<long long>(rows));
+  if (k < 1 || k > 2048) return fail(SI_ERR_INVALID_ARGUMENT, "1 <= k <= 2048 (got %d)", k);
+  if (rows == 0) return SI_OK;
+  if (!idx || !score) return fail(SI_ERR_INVALID_ARGUMENT, "idx and score must be non-null");
+  if (!aligned(idx, 4) || !aligned(score, 4))
+    return fail(SI_ERR_INVALID_ARGUMENT, "idx and score must be 4-byte aligned");
+  return launch_row_sort(idx, score, rows, k, static_cast<cudaStream_t>(stream));
 }
 
 si_status si_indexer_topk(const void* q, const void* kc, const float* w, int B, int S, int T,
@@ -161,6 +176,7 @@ si_status si_test_stream_timeout(const void* q, const void* kc, const float* w, 
   cfg.kc_scale = nullptr;
   cfg.wait_limit_ns = wait_limit_ns;
   cfg.test_withhold = 1;
+  cfg.unsorted = false;
   return launch_stream_topk(q, kc, w, B, S, T, 64, 128, m, k, out_idx, nullptr,
                             static_cast<cudaStream_t>(stream), cfg);
 }
@@ -219,6 +235,6 @@ const char* si_status_string(si_status s) {
 
 const char* si_last_error(void) { return g_last_error; }
 
-int si_version(void) { return 100; }
+int si_version(void) { return 200; }
 
 }  // extern "C"

@@ -38,7 +38,11 @@ struct StreamConfig {
   const float* kc_scale;
   uint64_t wait_limit_ns;
   int test_withhold;  // test hook: withhold one key-tile load (timeout path)
+  bool unsorted;      // leave rows in pool order (no in-kernel sort either)
 };
+
+// Sorts rows [rows, k] of (idx, score) in place by (score desc, index asc).
+si_status launch_row_sort(int32_t* idx, float* score, long long rows, int k, cudaStream_t stream);
 
 // Shared-memory plan of the streaming kernel for (k, key_tile, fp8); returns
 // false when it cannot fit.

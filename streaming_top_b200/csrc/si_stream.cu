@@ -20,11 +20,13 @@
 //                       columns) so the MMA of tile j+1 overlaps the
 //                       epilogue of tile j.
 //   warps 8..15         scoring.  Warp = TMEM lane quadrant (warp % 4, 32
-//                       keys) x 2 of the 4 queries.  tcgen05.ld 16x256b gives
-//                       a thread 4 keys x 16 heads of a query; ReLU and the
-//                       w-weighted head sum run in registers (w held in
-//                       registers for the whole unit), a 2-step shuffle
-//                       reduce-scatter leaves each thread one key's score.
+//                       keys) x 2 of the 4 queries.  tcgen05.ld 32x32b gives
+//                       each thread one key's 64 head logits per query (the
+//                       32-lane shape drains TMEM several times faster than
+//                       the 16-lane ones); the accumulator is released as
+//                       soon as it is in registers.  ReLU and the w-weighted
+//                       head sum run in registers, w read from a per-warp
+//                       shared-memory table by broadcast loads.
 //                       Causal mask, then threshold early-reject: a key is
 //                       appended to its query's candidate pool only if its
 //                       score beats the threshold the manager last
@@ -70,6 +72,9 @@ constexpr int N_SCORE_WARPS = 8;
 constexpr int HIST_BINS = 256;
 constexpr int N_AREAS = 2;         // append areas (double buffered)
 constexpr int CTRL_BYTES = 1024;
+// Head weights of the current unit, one private copy per scoring warp (its
+// two queries x 64 heads, fp32).
+constexpr int WTAB_BYTES = N_SCORE_WARPS * 2 * 64 * 4;
 // Register budgets: launched at 128 per thread (512 threads); warpgroup 0
 // (producer, MMA) and warpgroup 1 (managers) give registers to the two
 // scoring warpgroups: 128 * 40 + 128 * 120 + 256 * 176 = 65536.
@@ -109,6 +114,7 @@ struct Params {
   int n_stages;
   uint64_t wait_limit_ns;
   int test_withhold;
+  int sort_rows;          // finalize sorts each row itself (no scores to sort by later)
 };
 
 struct Unit {
@@ -168,36 +174,49 @@ __device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, f
 
 __device__ __forceinline__ float relu_u(uint32_t x) { return fmaxf(__uint_as_float(x), 0.f); }
 
-// One query's scores for the thread's key.  va / vb: 16x256b.x8 loads of the
-// quadrant's lanes 0-15 and 16-31: register 4r+e holds (key t1, head
-// 8r+2t0+e), register 4r+2+e holds (key t1+8, same head), where t0 = lane%4,
-// t1 = lane/4; vb likewise for keys t1+16, t1+24.  wq[2r+e] = w of head
-// 8r+2t0+e.  The four lanes sharing t1 reduce-scatter their 16-head partial
-// sums so that lane t0 ends with the full sum of key t1 + 8*t0.
-__device__ __forceinline__ float score_query(const uint32_t (&va)[32], const uint32_t (&vb)[32],
-                                             const float (&wq)[16], int lane) {
-  float s[4][2];
+// One query's score for the thread's key: x holds the key's 64 head logits
+// (a 32x32b TMEM load: thread = key, register = head), w the query's 64 head
+// weights in shared memory (every lane reads the same address: broadcast).
+// Four independent packed-FMA chains of 8 steps each.
+__device__ __forceinline__ float score_key(const uint32_t (&x)[64], const float* w) {
+  float a[4][2];
 #pragma unroll
-  for (int j = 0; j < 4; ++j) s[j][0] = s[j][1] = 0.f;
+  for (int c = 0; c < 4; ++c) a[c][0] = a[c][1] = 0.f;
+  const float4* w4 = reinterpret_cast<const float4*>(w);
 #pragma unroll
-  for (int r = 0; r < 8; ++r) {
-    const float w0 = wq[2 * r], w1 = wq[2 * r + 1];
-    fma2(s[0][0], s[0][1], w0, w1, relu_u(va[4 * r + 0]), relu_u(va[4 * r + 1]));
-    fma2(s[1][0], s[1][1], w0, w1, relu_u(va[4 * r + 2]), relu_u(va[4 * r + 3]));
-    fma2(s[2][0], s[2][1], w0, w1, relu_u(vb[4 * r + 0]), relu_u(vb[4 * r + 1]));
-    fma2(s[3][0], s[3][1], w0, w1, relu_u(vb[4 * r + 2]), relu_u(vb[4 * r + 3]));
+  for (int c = 0; c < 16; ++c) {
+    const float4 wv = w4[c];
+    fma2(a[c & 3][0], a[c & 3][1], wv.x, wv.y, relu_u(x[4 * c]), relu_u(x[4 * c + 1]));
+    fma2(a[(c + 2) & 3][0], a[(c + 2) & 3][1], wv.z, wv.w, relu_u(x[4 * c + 2]), relu_u(x[4 * c + 3]));
   }
-  const float p0 = s[0][0] + s[0][1], p1 = s[1][0] + s[1][1];
-  const float p2 = s[2][0] + s[2][1], p3 = s[3][0] + s[3][1];
-  const bool b0 = lane & 1, b1 = (lane >> 1) & 1;
-  // step 1: keep keys {b0, b0 + 2}, hand the other two to lane ^ 1
-  const float k0 = b0 ? p1 : p0, k1 = b0 ? p3 : p2;
-  const float g0 = b0 ? p0 : p1, g1 = b0 ? p2 : p3;
-  const float r0 = k0 + __shfl_xor_sync(0xFFFFFFFFu, g0, 1);
-  const float r1 = k1 + __shfl_xor_sync(0xFFFFFFFFu, g1, 1);
-  // step 2: keep key b0 + 2*b1
-  const float keep = b1 ? r1 : r0, give = b1 ? r0 : r1;
-  return keep + __shfl_xor_sync(0xFFFFFFFFu, give, 2);
+  return ((a[0][0] + a[0][1]) + (a[1][0] + a[1][1])) + ((a[2][0] + a[2][1]) + (a[3][0] + a[3][1]));
+}
+
+// The same with the query's 64 head weights in registers.
+__device__ __forceinline__ float score_key_regs(const uint32_t (&x)[64], const float (&w)[64]) {
+  float a[4][2];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) a[c][0] = a[c][1] = 0.f;
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {
+    fma2(a[c & 3][0], a[c & 3][1], w[4 * c], w[4 * c + 1], relu_u(x[4 * c]), relu_u(x[4 * c + 1]));
+    fma2(a[(c + 2) & 3][0], a[(c + 2) & 3][1], w[4 * c + 2], w[4 * c + 3], relu_u(x[4 * c + 2]),
+         relu_u(x[4 * c + 3]));
+  }
+  return ((a[0][0] + a[0][1]) + (a[1][0] + a[1][1])) + ((a[2][0] + a[2][1]) + (a[3][0] + a[3][1]));
+}
+
+// Appends the thread's key to its warp's segment when it passes the filter
+// (saddr: the segment's shared-memory address; n: entries so far, warp-uniform).
+__device__ __forceinline__ void seg_append(bool pass, uint32_t ord, uint32_t low, uint32_t saddr,
+                                           uint32_t& n, uint32_t lanemask) {
+  const uint32_t bal = __ballot_sync(0xFFFFFFFFu, pass);
+  if (pass) {
+    const uint64_t key = (static_cast<uint64_t>(ord) << 32) | low;
+    asm volatile("st.shared.u64 [%0], %1;" ::"r"(saddr + 8u * (n + __popc(bal & lanemask))), "l"(key)
+                 : "memory");
+  }
+  n += __popc(bal);
 }
 
 // Shared-memory layout (offsets from a 1024-byte aligned base).
@@ -217,7 +236,7 @@ __host__ __device__ constexpr int pool_stride(int cap, int seg_cap) {
 }
 
 struct Smem {
-  uint32_t q, kc, pool, hist, ctrl;
+  uint32_t q, kc, pool, hist, wtab, ctrl;
 };
 
 __host__ __device__ inline Smem carve(int n_stages, int cap, int seg_cap, int q_bytes, int kc_bytes) {
@@ -226,7 +245,8 @@ __host__ __device__ inline Smem carve(int n_stages, int cap, int seg_cap, int q_
   s.kc = q_bytes;
   s.pool = s.kc + n_stages * kc_bytes;
   s.hist = s.pool + QT * pool_stride(cap, seg_cap) * 8;
-  s.ctrl = s.hist + QT * HIST_BINS * 4;
+  s.wtab = s.hist + QT * HIST_BINS * 4;
+  s.ctrl = s.wtab + WTAB_BYTES;
   return s;
 }
 
@@ -262,6 +282,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint8_t* kc_s = smem + so.kc;
   uint64_t* pools = reinterpret_cast<uint64_t*>(smem + so.pool);
   uint32_t* hist = reinterpret_cast<uint32_t*>(smem + so.hist);
+  float* wtab = reinterpret_cast<float*>(smem + so.wtab);
   Ctrl* C = reinterpret_cast<Ctrl*>(smem + so.ctrl);
   volatile int* abort = &C->abort;
 
@@ -467,49 +488,66 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (!ok && lane == 0) st->cnt = 0;  // after an abort: contents unspecified
         __syncwarp();
         const size_t ob = (static_cast<size_t>(U.b) * p.S + t) * static_cast<size_t>(k);
-        topk::finalize(st, pool, qh, k, p.out_idx + ob, p.out_score ? p.out_score + ob : nullptr, lane);
+        topk::finalize(st, pool, qh, k, p.out_idx + ob, p.out_score ? p.out_score + ob : nullptr,
+                       p.sort_rows != 0, lane);
       }
     }
   } else {
     regs_inc<REGS_SCORE>();
     // ------------------------------------------------------------ scoring warps
     const int quad = warp & 3;        // TMEM lanes 32*quad .. 32*quad+31
-    const int qp = (warp - 8) >> 2;   // this warp's queries: 2*qp, 2*qp+1
-    const int t0 = lane & 3, t1 = lane >> 2;
-    const int key_off = quad * 32 + t1 + 8 * t0;  // key (within the tile) this lane scores
+    const int qp = (warp - 8) >> 2;   // this warp's queries: 2*qp (weights in registers), 2*qp+1 (table)
+    const int key_off = quad * 32 + lane;  // key (within the tile) this lane scores
+    float* wt = wtab + (warp - 8) * (2 * HEADS);
+    const uint32_t lanemask = (1u << lane) - 1u;
     const bool half_parts = p.key_tile < KT;
-    const int part_tiles = sub_tiles(p.key_tile);  // tiles per hand-off
-    const int n_phase = half_parts ? 2 : 1;
+    const int part_tiles = sub_tiles(p.key_tile);  // tiles per hand-off (key_tile >= 128)
+    // this warp's append segments in area 0 (area 1 is area_step bytes further)
+    const uint32_t seg_q0 = smem_u32(pools) + 8u * static_cast<uint32_t>((2 * qp) * stride + p.cap + quad * seg_cap);
+    const uint32_t seg_q1 = seg_q0 + 8u * static_cast<uint32_t>(stride);
+    const uint32_t area_step = 8u * 4u * static_cast<uint32_t>(seg_cap);
     uint32_t acc = 0, accph = 0, gp = 0;
+    bool ok = !*abort;
     for (int i = 0;; ++i) {
       const int u = unit_of(i, n_units);
       if (u < 0) break;
       const Unit U = decode_unit(u, p);
       if (U.n_kt == 0) continue;
-      // w of this lane's 16 heads (8r + 2*t0 + e) for both queries
-      float wq[2][16];
+      // the two queries' head weights (times the q scales for fp8) into this
+      // warp's table, 0 for queries past the end of the sequence; the first
+      // query's then go to registers
+      __syncwarp();
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int x = r * 32 + lane;
+        const int t = U.t0 + 2 * qp + (x >> 6);
+        float wv = 0.f;
+        if (t < p.S) {
+          const size_t wi = (static_cast<size_t>(U.b) * p.S + t) * HEADS + (x & 63);
+          wv = p.w[wi];
+          if (OPB == 1) wv *= p.q_scale[wi];
+        }
+        wt[x] = wv;
+      }
+      __syncwarp();
+      float w0[64];
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const float4 v = reinterpret_cast<const float4*>(wt)[c];
+        w0[4 * c] = v.x;
+        w0[4 * c + 1] = v.y;
+        w0[4 * c + 2] = v.z;
+        w0[4 * c + 3] = v.w;
+      }
       int nvis[2];
 #pragma unroll
       for (int qi = 0; qi < 2; ++qi) {
         const int t = U.t0 + 2 * qp + qi;
         const int n = t < p.S ? (t + 1) / p.m : 0;
         nvis[qi] = n < p.T ? n : p.T;
-        const size_t wb = (static_cast<size_t>(U.b) * p.S + (t < p.S ? t : p.S - 1)) * HEADS;
-#pragma unroll
-        for (int r = 0; r < 8; ++r) {
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int h = 8 * r + 2 * t0 + e;
-            float wv = p.w[wb + h];
-            if (OPB == 1) wv *= p.q_scale[wb + h];
-            wq[qi][2 * r + e] = t < p.S ? wv : 0.f;
-          }
-        }
       }
-      uint32_t thr_r[2] = {0u, 0u};
-      uint32_t seg_n[2] = {0u, 0u};
-      uint64_t* seg_ptr[2] = {pools, pools};
-      bool ok = !*abort;
+      uint32_t thr0 = 0u, thr1 = 0u, n0 = 0u, n1 = 0u;
+      int sub_pos = 0;
       for (int j = 0; j < U.n_kt; ++j) {
         ok = ok && !*abort;
         if (ok && !mbar_wait_bounded(&C->t_full[acc], accph, abort, p.wait_limit_ns)) {
@@ -517,71 +555,67 @@ __global__ void __launch_bounds__(THREADS, 1)
           ok = false;
         }
         const int s = j * KT + key_off;
-        uint32_t ord[2] = {0u, 0u};
+        uint32_t ord0 = 0u, ord1 = 0u;
         if (ok) {
           tc_fence_after();
           const uint32_t ta = tmem + (static_cast<uint32_t>(quad * 32) << 16) + acc * NCOLS + (2 * qp) * HEADS;
           float ksc = 1.f;
           if (OPB == 1 && s < p.T) ksc = p.kc_scale[static_cast<size_t>(U.b) * p.T + s];
-#pragma unroll
-          for (int qi = 0; qi < 2; ++qi) {
-            uint32_t va[32], vb[32];
-            tmem_ld_16x256b_x8(ta + qi * HEADS, va);
-            tmem_ld_16x256b_x8(ta + (16u << 16) + qi * HEADS, vb);
+          {
+            uint32_t x[64];
+            tmem_ld32_x64(ta, x);
             tmem_ld_wait();
-            ord[qi] = f32_ord(score_query(va, vb, wq[qi], lane) * ksc);
+            ord0 = f32_ord(score_key_regs(x, w0) * ksc);
           }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&C->t_empty[acc]);  // accumulator may be overwritten now
-#pragma unroll
-          for (int qi = 0; qi < 2; ++qi) {  // adopt the manager's latest threshold for this unit
-            const uint64_t pv = *reinterpret_cast<volatile uint64_t*>(&C->pub[2 * qp + qi]);
-            if (static_cast<int>(pv >> 32) == i) thr_r[qi] = max(thr_r[qi], static_cast<uint32_t>(pv));
+          {
+            uint32_t x[64];
+            tmem_ld32_x64(ta + HEADS, x);
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&C->t_empty[acc]);  // the logits are in registers now
+            ord1 = f32_ord(score_key(x, wt + HEADS) * ksc);
           }
+          // adopt the managers' latest thresholds for this unit
+          const uint64_t pv0 = *reinterpret_cast<volatile uint64_t*>(&C->pub[2 * qp]);
+          const uint64_t pv1 = *reinterpret_cast<volatile uint64_t*>(&C->pub[2 * qp + 1]);
+          if (static_cast<int>(pv0 >> 32) == i) thr0 = max(thr0, static_cast<uint32_t>(pv0));
+          if (static_cast<int>(pv1 >> 32) == i) thr1 = max(thr1, static_cast<uint32_t>(pv1));
         }
         if (++acc == 2) {
           acc = 0;
           accph ^= 1u;
         }
         const uint32_t low = static_cast<uint32_t>(~static_cast<uint32_t>(s));
-        for (int ph = 0; ph < n_phase; ++ph) {
-          const int a = gp & 1;
-          const bool starts = half_parts || (j % part_tiles == 0);
-          if (starts) {
+        const bool p0 = ok && s < nvis[0] && ord0 > thr0;
+        const bool p1 = ok && s < nvis[1] && ord1 > thr1;
+        // hand-offs: sub-partitions of part_tiles tiles (two per tile of 64-key partitions)
+        const int n_ho = half_parts ? 2 : 1;
+        for (int ph = 0; ph < n_ho; ++ph) {
+          const uint32_t a = gp & 1u;
+          if (half_parts || sub_pos == 0) {
             // open an append area: wait until its manager has merged its last use
-            const uint32_t use = gp >> 1;
-            if (ok && !mbar_wait_bounded(&C->seg_free[a][qp], (use & 1u) ^ 1u, abort, p.wait_limit_ns)) {
+            if (ok && !mbar_wait_bounded(&C->seg_free[a][qp], ((gp >> 1) & 1u) ^ 1u, abort, p.wait_limit_ns)) {
               record_error(p, abort, ERR_WAIT_SEG_FREE);
               ok = false;
             }
-#pragma unroll
-            for (int qi = 0; qi < 2; ++qi) {
-              seg_n[qi] = 0u;
-              seg_ptr[qi] = pools + (2 * qp + qi) * stride + p.cap + (a * 4 + quad) * seg_cap;
-            }
+            n0 = n1 = 0u;
           }
-          if (ok && (!half_parts || (quad >> 1) == ph)) {
-#pragma unroll
-            for (int qi = 0; qi < 2; ++qi) {
-              const bool pq = s < nvis[qi] && ord[qi] > thr_r[qi];
-              const uint32_t bal = __ballot_sync(0xFFFFFFFFu, pq);
-              if (pq)
-                seg_ptr[qi][seg_n[qi] + __popc(bal & ((1u << lane) - 1u))] =
-                    (static_cast<uint64_t>(ord[qi]) << 32) | low;
-              seg_n[qi] += __popc(bal);
-            }
+          if (!half_parts || (quad >> 1) == ph) {
+            seg_append(p0 && ok, ord0, low, seg_q0 + a * area_step, n0, lanemask);
+            seg_append(p1 && ok, ord1, low, seg_q1 + a * area_step, n1, lanemask);
           }
-          const bool ends = half_parts || ((j + 1) % part_tiles == 0) || (j == U.n_kt - 1);
+          const bool ends = half_parts || sub_pos == part_tiles - 1 || j == U.n_kt - 1;
           if (ends) {
             __syncwarp();
             if (lane == 0) {
-              C->seg_cnt[a][2 * qp][quad] = seg_n[0];
-              C->seg_cnt[a][2 * qp + 1][quad] = seg_n[1];
+              C->seg_cnt[a][2 * qp][quad] = n0;
+              C->seg_cnt[a][2 * qp + 1][quad] = n1;
               mbar_arrive(&C->seg_done[a][qp]);  // release: this warp's appends are visible
             }
             ++gp;
           }
+          if (!half_parts) sub_pos = ends ? 0 : sub_pos + 1;
         }
       }
     }
@@ -611,7 +645,7 @@ bool stream_smem_plan(int k, int key_tile, int fp8, int* n_stages, int* pool_cap
   const size_t limit = 227 * 1024;
   const size_t areas = static_cast<size_t>(QT) * N_AREAS * 4 * seg_cap * 8;
   for (int ns = 4; ns >= 2; --ns) {
-    const size_t fixed = q_bytes + ns * kc_bytes + areas + QT * HIST_BINS * 4 + CTRL_BYTES +
+    const size_t fixed = q_bytes + ns * kc_bytes + areas + QT * HIST_BINS * 4 + WTAB_BYTES + CTRL_BYTES +
                          1024 /* alignment slack */;
     if (fixed >= limit) continue;
     const int cap_max = static_cast<int>((limit - fixed) / (QT * 8));
@@ -676,6 +710,9 @@ si_status launch_stream_topk(const void* q, const void* kc, const float* w, int 
   p.n_stages = n_stages;
   p.wait_limit_ns = cfg.wait_limit_ns;
   p.test_withhold = cfg.test_withhold;
+  // with scores stored, the rows are sorted afterwards by a separate pass
+  // over the output; without them the managers sort before storing
+  p.sort_rows = (!cfg.unsorted && out_score == nullptr) ? 1 : 0;
 
   // chunk driver: one persistent launch per chunk of queries
   const int n_qt_total = (S + QT - 1) / QT;

@@ -134,7 +134,7 @@ __device__ __forceinline__ int pool_compact(uint64_t* pool, int n, uint32_t thr,
 // return the orderable score of the k-th.  Radix select, most significant
 // digit first, beginning below the bits all keys share; 8-bit digits.
 // hist (256 words) is scratch.  One warp.
-__device__ uint32_t pool_select(uint64_t* pool, int n, int k, uint32_t* hist, int lane) {
+__device__ inline uint32_t pool_select(uint64_t* pool, int n, int k, uint32_t* hist, int lane) {
   uint64_t vor = 0, vand = ~0ull;
   for (int i = lane; i < n; i += 32) {
     const uint64_t x = pool[i];
@@ -374,7 +374,7 @@ __device__ __forceinline__ void merge(QState* st, uint64_t* pool, const uint64_t
 //    exactly k by radix select and refit.
 // Invariant: every processed key that can still be in the final top-k is in
 // the pool, and once thr > 0 at least k entries have orderable score >= thr.
-__device__ void refresh(QState* st, uint64_t* pool, uint32_t* hist, int k, int cap, int room,
+__device__ inline void refresh(QState* st, uint64_t* pool, uint32_t* hist, int k, int cap, int room,
                         int lane) {
   int n = static_cast<int>(st->cnt);
   uint32_t thr = st->thr, base = st->base, shift = st->shift;
@@ -433,14 +433,15 @@ __device__ void refresh(QState* st, uint64_t* pool, uint32_t* hist, int k, int c
   __syncwarp();
 }
 
-// Final step for one query: exactly the k best pool entries, sorted by
-// (score desc, index asc), stored to out_idx / out_score ([k] each; -1 /
-// -inf after the valid ones).  With a histogram, one pass keeps the entries
+// Final step for one query: exactly the k best pool entries, stored to
+// out_idx / out_score ([k] each; -1 / -inf after the valid ones), sorted by
+// (score desc, index asc) when `sort`, else in pool order (a later pass over
+// the stored rows sorts them).  With a histogram, one pass keeps the entries
 // of the bins above the k-th's bin and gathers that boundary bin's entries
 // (into the histogram's memory, when they fit: 128 entries), a small sort
 // picks the boundary keys still needed; otherwise radix select.  One warp.
-__device__ void finalize(QState* st, uint64_t* pool, uint32_t* hist, int k, int32_t* out_idx,
-                         float* out_score, int lane) {
+__device__ inline void finalize(QState* st, uint64_t* pool, uint32_t* hist, int k, int32_t* out_idx,
+                         float* out_score, bool sort, int lane) {
   int n = static_cast<int>(st->cnt);
   if (n > k) {
     bool done = false;
@@ -506,7 +507,7 @@ __device__ void finalize(QState* st, uint64_t* pool, uint32_t* hist, int k, int3
       n = k;
     }
   }
-  pool_sort(pool, n, lane);
+  if (sort) pool_sort(pool, n, lane);
   for (int x = lane; x < k; x += 32) {
     int32_t id = -1;
     float sc = -__int_as_float(0x7f800000);

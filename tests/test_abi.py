@@ -85,3 +85,16 @@ def test_workspace_size():
     assert si.workspace_size(1, 1024, 256, 64, 128, 4, 64, materialize=False) == 0
     need = si.workspace_size(1, 1024, 256, 64, 128, 4, 64, materialize=True)
     assert need >= 4 * 1024 * 256 * 65
+
+
+@pytest.mark.parametrize("idx,score,rows,k,status", [
+    (P, P, 4, 0, si.SI_ERR_INVALID_ARGUMENT),
+    (P, P, 4, 4096, si.SI_ERR_INVALID_ARGUMENT),
+    (P, P, -1, 8, si.SI_ERR_INVALID_ARGUMENT),
+    (None, P, 4, 8, si.SI_ERR_INVALID_ARGUMENT),
+    (P, None, 4, 8, si.SI_ERR_INVALID_ARGUMENT),
+    (P + 2, P, 4, 8, si.SI_ERR_INVALID_ARGUMENT),
+    (None, None, 0, 8, si.SI_OK),  # nothing to sort: no device work at all
+])
+def test_row_sort_validation(idx, score, rows, k, status):
+    assert si.lib().si_sort_topk_rows(idx, score, rows, k, None) == status

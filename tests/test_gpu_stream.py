@@ -244,3 +244,61 @@ def test_unsupported_shapes_are_refused():
     with pytest.raises(si.SIError) as e:
         si.indexer_topk(q, kc, w, 4, 8)
     assert e.value.status == si.SI_ERR_UNSUPPORTED
+
+
+# ------------------------------------------------------------ output ordering
+def test_unsorted_option_gives_the_same_rows():
+    """unsorted=True: each row holds the same entries, valid ones first; the
+    row sort entry point then restores the default order exactly."""
+    inp = _int_inputs(1, 2048, 512, seed=31)
+    q, kc, w = _dev(inp)
+    k = 200
+    si_idx, si_sc = si.indexer_topk(q, kc, w, 4, k)
+    ui, us = si.indexer_topk(q, kc, w, 4, k, unsorted=True)
+    assert si.device_status() == si.SI_OK
+    a_i, a_s = si_idx.cpu().numpy().reshape(-1, k), si_sc.cpu().numpy().reshape(-1, k)
+    b_i, b_s = ui.cpu().numpy().reshape(-1, k), us.cpu().numpy().reshape(-1, k)
+    for r in range(a_i.shape[0]):
+        nv = int((a_i[r] >= 0).sum())
+        assert np.all(b_i[r, :nv] >= 0) and np.all(b_i[r, nv:] == -1)
+        assert sorted(zip(a_i[r, :nv], a_s[r, :nv])) == sorted(zip(b_i[r, :nv], b_s[r, :nv]))
+    si.sort_topk_rows(ui, us)
+    assert si.device_status() == si.SI_OK
+    assert np.array_equal(ui.cpu().numpy().reshape(-1, k), a_i)
+    assert np.array_equal(us.cpu().numpy().reshape(-1, k), a_s)
+
+
+def test_without_scores_rows_come_sorted():
+    """out_score omitted: the kernel sorts each row itself before storing."""
+    inp = _int_inputs(1, 2048, 512, seed=32)
+    q, kc, w = _dev(inp)
+    for k in (64, 300, 512):
+        gi, gs = si.indexer_topk(q, kc, w, 4, k, with_score=False)
+        assert gs is None and si.device_status() == si.SI_OK
+        oi, _, _ = oracle.topk(inp["q"], inp["kc"], inp["w"], 4, k)
+        assert np.array_equal(gi.cpu().numpy().reshape(-1, k), oi)
+
+
+@pytest.mark.parametrize("k", [1, 7, 64, 100, 512, 1000, 2048])
+def test_row_sort_matches_lexicographic_order(k):
+    """si_sort_topk_rows on arbitrary rows: score descending, index ascending,
+    (-1, -inf) padding last; -0.0 ranks with +0.0."""
+    rng = np.random.default_rng(k)
+    rows = 300
+    idx = rng.permutation(rows * k).astype(np.int32).reshape(rows, k)
+    sc = rng.choice(np.float32([-2.5, -0.0, 0.0, 1.0, 1.0, 3.25, 7.0]), size=(rows, k))
+    sc += rng.integers(0, 3, size=(rows, k)).astype(np.float32) * (rng.random((rows, k)) < 0.5)
+    pad = rng.random((rows, k)) < 0.1
+    idx[pad] = -1
+    sc[pad] = -np.inf
+    ti, ts = torch.from_numpy(idx).cuda(), torch.from_numpy(sc).cuda()
+    si.sort_topk_rows(ti, ts)
+    assert si.device_status() == si.SI_OK
+    gi, gs = ti.cpu().numpy(), ts.cpu().numpy()
+    for r in range(rows):
+        # padding sorts last: give it the lowest rank explicitly
+        s = np.where(idx[r] < 0, -np.inf, sc[r]).astype(np.float64) + 0.0  # -0.0 -> 0.0
+        key_idx = np.where(idx[r] < 0, np.iinfo(np.int64).max, idx[r].astype(np.int64))
+        order = np.lexsort((key_idx, -s))
+        assert np.array_equal(gi[r], idx[r][order]), r
+        assert np.array_equal(np.abs(gs[r]), np.abs(sc[r][order])), r
