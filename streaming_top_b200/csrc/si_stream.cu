@@ -25,22 +25,25 @@
 //                       32-lane shape drains TMEM several times faster than
 //                       the 16-lane ones); the accumulator is released as
 //                       soon as it is in registers.  ReLU and the w-weighted
-//                       head sum run in registers, w read from a per-warp
-//                       shared-memory table by broadcast loads.
-//                       Causal mask, then threshold early-reject: a key is
-//                       appended to its query's candidate pool only if its
-//                       score beats the threshold the manager last
-//                       published; appends go to the warp's private segment
-//                       of a double-buffered append area.
-//   warps 4..7          top-k managers, one per query: they merge each
-//                       hand-off of candidates into the query's running pool
-//                       and count them into a 256-bin histogram of its
-//                       scores; at the end of every partition of `key_tile`
-//                       keys (the pages' key tile) they raise and publish
-//                       the threshold and compact the pool when it fills; at
-//                       the end of the unit they select the exact k best,
-//                       sort them and store them -- while the scoring warps
-//                       already work on the next unit.
+//                       head sum run in registers: one query's weights sit in
+//                       registers, the other's are read from a per-warp
+//                       shared-memory table by broadcast loads.  Causal mask,
+//                       then threshold early-reject: a key becomes a
+//                       candidate only if its score beats the threshold its
+//                       manager last published; each warp compacts its
+//                       candidates into its segment of a slot of a ring of
+//                       per-tile candidate buffers.
+//   warps 4..7          top-k managers, one per query: per tile they move the
+//                       query's candidates from the ring slot into the
+//                       query's running pool and count them into a 256-bin
+//                       histogram of its scores; at the end of every
+//                       partition of `key_tile` keys (the pages' key tile)
+//                       they raise and publish the threshold and compact the
+//                       pool when it fills; at the end of the unit they
+//                       select the exact k best and store them (sorted only
+//                       when no scores are stored; otherwise a row-sort pass
+//                       orders the rows) -- while the scoring warps already
+//                       work on the next unit.
 //   warps 2, 3          idle (they complete warpgroup 0).
 //
 // Keys are packed as (orderable fp32 score << 32) | ~index, so one unsigned
@@ -70,7 +73,10 @@ constexpr int NCOLS = QT * HEADS;  // 256 = MMA N
 constexpr int THREADS = 512;       // 16 warps
 constexpr int N_SCORE_WARPS = 8;
 constexpr int HIST_BINS = 256;
-constexpr int N_AREAS = 2;         // append areas (double buffered)
+// Candidate ring between scorers and managers: per slot (one key tile) and
+// query, one segment of up to 32 candidates per TMEM lane quadrant.
+constexpr int RING = 4;
+constexpr int RING_BYTES = RING * QT * 4 * 32 * 8;
 constexpr int CTRL_BYTES = 1024;
 // Head weights of the current unit, one private copy per scoring warp (its
 // two queries x 64 heads, fp32).
@@ -83,22 +89,10 @@ constexpr uint32_t REGS_MGR = 120;
 constexpr uint32_t REGS_SCORE = 176;
 static_assert(128 * REGS_PIPE + 128 * REGS_MGR + 256 * REGS_SCORE <= 512 * 128, "register split");
 
-// Scoring warps hand their candidates to the managers in sub-partitions of
-// at most 256 keys (a 64-key partition is half a tile, otherwise 1 or 2
-// tiles); the managers refresh the threshold once per partition.
-__host__ __device__ constexpr int sub_keys(int key_tile) {
-  return key_tile <= 256 ? key_tile : (key_tile % 256 == 0 ? 256 : 128);
-}
-__host__ __device__ constexpr int sub_tiles(int key_tile) {
-  return sub_keys(key_tile) >= KT ? sub_keys(key_tile) / KT : 1;
-}
-// Appends one scoring warp can make to one query's pool in one
-// sub-partition: 32 keys per 128-key tile.
-__host__ __device__ constexpr int seg_capacity(int key_tile) { return 32 * sub_tiles(key_tile); }
 
 enum { ERR_WAIT_Q = 1, ERR_WAIT_KC = 2, ERR_WAIT_TMEM_EMPTY = 3, ERR_WAIT_TMEM_FULL = 4,
-       ERR_WAIT_QFREE = 5, ERR_WAIT_KFREE = 6, ERR_WAIT_DRAIN = 7, ERR_WAIT_SEG_FREE = 8,
-       ERR_WAIT_SEG_DONE = 9 };
+       ERR_WAIT_QFREE = 5, ERR_WAIT_KFREE = 6, ERR_WAIT_DRAIN = 7, ERR_WAIT_RING_FREE = 8,
+       ERR_WAIT_RING_FULL = 9 };
 
 struct Params {
   const float* w;         // [B,S,H]
@@ -140,12 +134,6 @@ __device__ __forceinline__ int unit_of(int i, int n_units) {
   if (base >= n_units) return -1;
   const long long u = base + ((i & 1) ? (G - 1 - c) : c);
   return u < n_units ? static_cast<int>(u) : -1;
-}
-
-__device__ __forceinline__ int n_subparts(const Unit& U, const Params& p) {
-  if (p.key_tile < KT) return 2 * U.n_kt;
-  const int st = sub_tiles(p.key_tile);
-  return (U.n_kt + st - 1) / st;
 }
 
 __device__ __forceinline__ uint32_t f32_ord(float f) {
@@ -206,19 +194,6 @@ __device__ __forceinline__ float score_key_regs(const uint32_t (&x)[64], const f
   return ((a[0][0] + a[0][1]) + (a[1][0] + a[1][1])) + ((a[2][0] + a[2][1]) + (a[3][0] + a[3][1]));
 }
 
-// Appends the thread's key to its warp's segment when it passes the filter
-// (saddr: the segment's shared-memory address; n: entries so far, warp-uniform).
-__device__ __forceinline__ void seg_append(bool pass, uint32_t ord, uint32_t low, uint32_t saddr,
-                                           uint32_t& n, uint32_t lanemask) {
-  const uint32_t bal = __ballot_sync(0xFFFFFFFFu, pass);
-  if (pass) {
-    const uint64_t key = (static_cast<uint64_t>(ord) << 32) | low;
-    asm volatile("st.shared.u64 [%0], %1;" ::"r"(saddr + 8u * (n + __popc(bal & lanemask))), "l"(key)
-                 : "memory");
-  }
-  n += __popc(bal);
-}
-
 // Shared-memory layout (offsets from a 1024-byte aligned base).
 template <int OPB>
 struct Layout {
@@ -229,39 +204,36 @@ struct Layout {
   static constexpr int N_MMA = DIM * OPB / 32;       // K steps of 32 bytes
 };
 
-// Per-query pool: main region [0, cap) then N_AREAS append areas of
-// 4 * seg_cap entries each.
-__host__ __device__ constexpr int pool_stride(int cap, int seg_cap) {
-  return cap + N_AREAS * 4 * seg_cap;
-}
-
 struct Smem {
-  uint32_t q, kc, pool, hist, wtab, ctrl;
+  uint32_t q, kc, pool, hist, ring, wtab, ctrl;
 };
 
-__host__ __device__ inline Smem carve(int n_stages, int cap, int seg_cap, int q_bytes, int kc_bytes) {
+// Per-query pools of `cap` entries, then the histograms, the candidate ring
+// ([slot][query][quadrant][32] packed keys), the weight tables and the
+// control block.
+__host__ __device__ inline Smem carve(int n_stages, int cap, int q_bytes, int kc_bytes) {
   Smem s;
   s.q = 0;
   s.kc = q_bytes;
   s.pool = s.kc + n_stages * kc_bytes;
-  s.hist = s.pool + QT * pool_stride(cap, seg_cap) * 8;
-  s.wtab = s.hist + QT * HIST_BINS * 4;
+  s.hist = s.pool + QT * cap * 8;
+  s.ring = s.hist + QT * HIST_BINS * 4;
+  s.wtab = s.ring + RING_BYTES;
   s.ctrl = s.wtab + WTAB_BYTES;
   return s;
 }
 
-// Control block (CTRL_BYTES): mbarriers, manager state, published
-// thresholds, segment counts, TMEM slot, abort flag.
+// Control block (CTRL_BYTES): mbarriers, manager state, TMEM slot, abort flag.
 struct Ctrl {
   uint64_t full[4], empty[4];
   uint64_t q_full, q_empty;
   uint64_t t_full[2], t_empty[2];
   uint64_t mma_done;
-  uint64_t seg_done[N_AREAS][2];  // [area][query pair]: scoring warps -> manager
-  uint64_t seg_free[N_AREAS][2];  // manager -> scoring warps
-  uint64_t pub[QT];               // (unit tag << 32) | threshold
+  uint64_t ring_full[RING];   // the 8 scoring warps have written the slot
+  uint64_t ring_free[RING];   // the 4 managers have read the slot
+  uint64_t pub[QT];           // (unit tag << 32) | threshold, published by the managers
   topk::QState qs[QT];
-  uint32_t seg_cnt[N_AREAS][QT][4];
+  uint32_t ring_cnt[RING][QT][4];
   uint32_t tmem_slot;
   int abort;
 };
@@ -275,13 +247,12 @@ __global__ void __launch_bounds__(THREADS, 1)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  const int seg_cap = seg_capacity(p.key_tile);
-  const int stride = pool_stride(p.cap, seg_cap);
-  const Smem so = carve(p.n_stages, p.cap, seg_cap, L::Q_BYTES, L::KC_BYTES);
+  const Smem so = carve(p.n_stages, p.cap, L::Q_BYTES, L::KC_BYTES);
   uint8_t* q_s = smem + so.q;
   uint8_t* kc_s = smem + so.kc;
   uint64_t* pools = reinterpret_cast<uint64_t*>(smem + so.pool);
   uint32_t* hist = reinterpret_cast<uint32_t*>(smem + so.hist);
+  uint64_t* ring = reinterpret_cast<uint64_t*>(smem + so.ring);
   float* wtab = reinterpret_cast<float*>(smem + so.wtab);
   Ctrl* C = reinterpret_cast<Ctrl*>(smem + so.ctrl);
   volatile int* abort = &C->abort;
@@ -300,11 +271,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&C->t_empty[b], N_SCORE_WARPS);
     }
     mbar_init(&C->mma_done, 1);
-    for (int a = 0; a < N_AREAS; ++a)
-      for (int g = 0; g < 2; ++g) {
-        mbar_init(&C->seg_done[a][g], 4);  // the 4 scoring warps of a query pair
-        mbar_init(&C->seg_free[a][g], 2);  // the pair's two managers
-      }
+    for (int r = 0; r < RING; ++r) {
+      mbar_init(&C->ring_full[r], N_SCORE_WARPS);
+      mbar_init(&C->ring_free[r], QT);
+    }
     for (int q = 0; q < QT; ++q) C->pub[q] = 0ull;
     *abort = 0;
     fence_mbar_init();
@@ -441,14 +411,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     regs_dec<REGS_MGR>();
     // ------------------------------------------------------------ top-k managers
     const int q = warp - 4;   // this manager's query in the unit
-    const int g = q >> 1;     // the query pair whose scoring warps feed it
     const int k = p.k;
     const int room = p.key_tile;  // appends one partition can bring
-    const int subs_per_part = p.key_tile / sub_keys(p.key_tile);
-    uint64_t* pool = pools + q * stride;
+    const int tpp = p.key_tile < KT ? 1 : p.key_tile / KT;  // tiles per partition
+    uint64_t* pool = pools + q * p.cap;
     uint32_t* qh = hist + q * HIST_BINS;
     topk::QState* st = &C->qs[q];
-    uint32_t gp = 0;          // hand-offs merged so far (CTA-wide numbering)
+    uint32_t tix = 0;         // score tiles consumed (ring position)
     bool ok = true;
     for (int i = 0;; ++i) {
       const int u = unit_of(i, n_units);
@@ -462,28 +431,36 @@ __global__ void __launch_bounds__(THREADS, 1)
         st->binned = 0;
       }
       __syncwarp();
-      const int np = n_subparts(U, p);
-      for (int pi = 0; pi < np; ++pi, ++gp) {
-        const int a = gp & 1;
-        const uint32_t use = gp >> 1;
-        if (ok && !*abort && !mbar_wait_bounded(&C->seg_done[a][g], use & 1u, abort, p.wait_limit_ns)) {
-          record_error(p, abort, ERR_WAIT_SEG_DONE);
+      const int t = U.t0 + q;
+      int in_part = 0;
+      for (int j = 0; j < U.n_kt; ++j, ++tix) {
+        const uint32_t slot = tix & (RING - 1), par = (tix / RING) & 1u;
+        if (ok && !*abort && !mbar_wait_bounded(&C->ring_full[slot], par, abort, p.wait_limit_ns)) {
+          record_error(p, abort, ERR_WAIT_RING_FULL);
           ok = false;
         }
         ok = ok && !*abort;
-        if (ok) {
-          topk::merge(st, pool, pool + p.cap + a * 4 * seg_cap, C->seg_cnt[a][q], seg_cap, qh, lane);
-          if (((pi + 1) % subs_per_part == 0) || (pi == np - 1)) {
+        const uint64_t* area = ring + (slot * QT + q) * 4 * 32;
+        if (ok && p.key_tile < KT) {
+          // 64-key partitions: quadrants 0-1 hold keys 0-63 of the tile, 2-3 the rest
+          topk::merge(st, pool, area, C->ring_cnt[slot][q], 32, qh, lane, 0, 2);
+          topk::refresh(st, pool, qh, k, p.cap, room, lane);
+          topk::merge(st, pool, area, C->ring_cnt[slot][q], 32, qh, lane, 2, 4);
+        } else if (ok) {
+          topk::merge(st, pool, area, C->ring_cnt[slot][q], 32, qh, lane);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&C->ring_free[slot]);  // the slot has been read
+        if (++in_part == tpp || j == U.n_kt - 1) {
+          in_part = 0;
+          if (ok) {
             topk::refresh(st, pool, qh, k, p.cap, room, lane);
             if (lane == 0)
               *reinterpret_cast<volatile uint64_t*>(&C->pub[q]) = (static_cast<uint64_t>(i) << 32) | st->thr;
           }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&C->seg_free[a][g]);
       }
       // finalize this unit's query while the scorers move on
-      const int t = U.t0 + q;
       if (t < p.S) {
         if (!ok && lane == 0) st->cnt = 0;  // after an abort: contents unspecified
         __syncwarp();
@@ -500,13 +477,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int key_off = quad * 32 + lane;  // key (within the tile) this lane scores
     float* wt = wtab + (warp - 8) * (2 * HEADS);
     const uint32_t lanemask = (1u << lane) - 1u;
-    const bool half_parts = p.key_tile < KT;
-    const int part_tiles = sub_tiles(p.key_tile);  // tiles per hand-off (key_tile >= 128)
-    // this warp's append segments in area 0 (area 1 is area_step bytes further)
-    const uint32_t seg_q0 = smem_u32(pools) + 8u * static_cast<uint32_t>((2 * qp) * stride + p.cap + quad * seg_cap);
-    const uint32_t seg_q1 = seg_q0 + 8u * static_cast<uint32_t>(stride);
-    const uint32_t area_step = 8u * 4u * static_cast<uint32_t>(seg_cap);
-    uint32_t acc = 0, accph = 0, gp = 0;
+    uint32_t acc = 0, accph = 0, tix = 0;
     bool ok = !*abort;
     for (int i = 0;; ++i) {
       const int u = unit_of(i, n_units);
@@ -546,9 +517,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int n = t < p.S ? (t + 1) / p.m : 0;
         nvis[qi] = n < p.T ? n : p.T;
       }
-      uint32_t thr0 = 0u, thr1 = 0u, n0 = 0u, n1 = 0u;
-      int sub_pos = 0;
-      for (int j = 0; j < U.n_kt; ++j) {
+      uint32_t thr0 = 0u, thr1 = 0u;
+      for (int j = 0; j < U.n_kt; ++j, ++tix) {
         ok = ok && !*abort;
         if (ok && !mbar_wait_bounded(&C->t_full[acc], accph, abort, p.wait_limit_ns)) {
           record_error(p, abort, ERR_WAIT_TMEM_FULL);
@@ -586,37 +556,26 @@ __global__ void __launch_bounds__(THREADS, 1)
           acc = 0;
           accph ^= 1u;
         }
-        const uint32_t low = static_cast<uint32_t>(~static_cast<uint32_t>(s));
+        // hand the tile's candidates (visible keys above the threshold) to the
+        // managers: this warp's segment of the ring slot, per query
+        const uint32_t slot = tix & (RING - 1), par = (tix / RING) & 1u;
+        if (ok && !mbar_wait_bounded(&C->ring_free[slot], par ^ 1u, abort, p.wait_limit_ns)) {
+          record_error(p, abort, ERR_WAIT_RING_FREE);
+          ok = false;
+        }
         const bool p0 = ok && s < nvis[0] && ord0 > thr0;
         const bool p1 = ok && s < nvis[1] && ord1 > thr1;
-        // hand-offs: sub-partitions of part_tiles tiles (two per tile of 64-key partitions)
-        const int n_ho = half_parts ? 2 : 1;
-        for (int ph = 0; ph < n_ho; ++ph) {
-          const uint32_t a = gp & 1u;
-          if (half_parts || sub_pos == 0) {
-            // open an append area: wait until its manager has merged its last use
-            if (ok && !mbar_wait_bounded(&C->seg_free[a][qp], ((gp >> 1) & 1u) ^ 1u, abort, p.wait_limit_ns)) {
-              record_error(p, abort, ERR_WAIT_SEG_FREE);
-              ok = false;
-            }
-            n0 = n1 = 0u;
-          }
-          if (!half_parts || (quad >> 1) == ph) {
-            seg_append(p0 && ok, ord0, low, seg_q0 + a * area_step, n0, lanemask);
-            seg_append(p1 && ok, ord1, low, seg_q1 + a * area_step, n1, lanemask);
-          }
-          const bool ends = half_parts || sub_pos == part_tiles - 1 || j == U.n_kt - 1;
-          if (ends) {
-            __syncwarp();
-            if (lane == 0) {
-              C->seg_cnt[a][2 * qp][quad] = n0;
-              C->seg_cnt[a][2 * qp + 1][quad] = n1;
-              mbar_arrive(&C->seg_done[a][qp]);  // release: this warp's appends are visible
-            }
-            ++gp;
-          }
-          if (!half_parts) sub_pos = ends ? 0 : sub_pos + 1;
+        const uint32_t b0 = __ballot_sync(0xFFFFFFFFu, p0), b1 = __ballot_sync(0xFFFFFFFFu, p1);
+        const uint32_t low = static_cast<uint32_t>(~static_cast<uint32_t>(s));
+        uint64_t* seg0 = ring + ((slot * QT + 2 * qp) * 4 + quad) * 32;
+        if (p0) seg0[__popc(b0 & lanemask)] = (static_cast<uint64_t>(ord0) << 32) | low;
+        if (p1) seg0[4 * 32 + __popc(b1 & lanemask)] = (static_cast<uint64_t>(ord1) << 32) | low;
+        if (lane == 0) {
+          C->ring_cnt[slot][2 * qp][quad] = __popc(b0);
+          C->ring_cnt[slot][2 * qp + 1][quad] = __popc(b1);
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&C->ring_full[slot]);  // release: the candidates are visible
       }
     }
   }
@@ -633,24 +592,21 @@ bool stream_smem_plan(int k, int key_tile, int fp8, int* n_stages, int* pool_cap
   const int opb = fp8 ? 1 : 2;
   int np2 = 32;
   while (np2 < k) np2 <<= 1;
-  const int seg_cap = seg_capacity(key_tile);
   const int room = key_tile;  // one partition's appends
-  // the main region takes a whole partition on top of k survivors, holds the
-  // padded final sort, and, when shared memory allows, up to k more so
-  // compaction stays rare
+  // the pool takes a whole partition on top of k survivors and holds the
+  // padded final sort; a larger pool makes compaction rarer, which is worth
+  // more than a third key-tile stage (the key tiles come from L2)
   const int cap_min = std::max(k + room, np2);
-  const int cap_want = std::max(cap_min, 2 * k + room);
+  const int cap_want = std::max(cap_min, 4 * k + room);
   const size_t q_bytes = static_cast<size_t>(NCOLS) * DIM * opb;
   const size_t kc_bytes = static_cast<size_t>(KT) * DIM * opb;
   const size_t limit = 227 * 1024;
-  const size_t areas = static_cast<size_t>(QT) * N_AREAS * 4 * seg_cap * 8;
-  for (int ns = 4; ns >= 2; --ns) {
-    const size_t fixed = q_bytes + ns * kc_bytes + areas + QT * HIST_BINS * 4 + WTAB_BYTES + CTRL_BYTES +
-                         1024 /* alignment slack */;
+  for (int ns = 3; ns >= 2; --ns) {
+    const size_t fixed = q_bytes + ns * kc_bytes + RING_BYTES + QT * HIST_BINS * 4 + WTAB_BYTES +
+                         CTRL_BYTES + 1024 /* alignment slack */;
     if (fixed >= limit) continue;
     const int cap_max = static_cast<int>((limit - fixed) / (QT * 8));
-    if (cap_max < cap_min) continue;
-    if (ns == 4 && cap_max < cap_want) continue;  // a larger pool beats a fourth stage
+    if (cap_max < cap_min || (ns > 2 && cap_max < cap_want)) continue;
     const int cap = std::min(cap_max, cap_want);
     *n_stages = ns;
     *pool_cap = cap;

@@ -335,12 +335,14 @@ __device__ __forceinline__ void pool_sort(uint64_t* pool, int n, int lane) {
   }
 }
 
-// merge(): move the query's candidates (four segments) to the end of its
+// merge(): move the query's candidates -- segments w_lo .. w_hi-1 of four,
+// segment w at area + w * seg_cap holding seg[w] entries -- to the end of its
 // main region in one pass over all lanes, counting them into the histogram
-// once it exists.
+// once it exists.  One warp.
 __device__ __forceinline__ void merge(QState* st, uint64_t* pool, const uint64_t* area,
-                                      const uint32_t* seg, int seg_cap, uint32_t* hist, int lane) {
-  const uint32_t c = lane < 4 ? seg[lane] : 0u;
+                                      const uint32_t* seg, int seg_cap, uint32_t* hist, int lane,
+                                      int w_lo = 0, int w_hi = 4) {
+  const uint32_t c = lane >= w_lo && lane < w_hi ? seg[lane] : 0u;
   const uint32_t c0 = __shfl_sync(0xFFFFFFFFu, c, 0), c1 = __shfl_sync(0xFFFFFFFFu, c, 1);
   const uint32_t c2 = __shfl_sync(0xFFFFFFFFu, c, 2), c3 = __shfl_sync(0xFFFFFFFFu, c, 3);
   const uint32_t o1 = c0, o2 = c0 + c1, o3 = c0 + c1 + c2, tot = o3 + c3;
@@ -348,7 +350,7 @@ __device__ __forceinline__ void merge(QState* st, uint64_t* pool, const uint64_t
   const bool binned = st->binned != 0;
   const uint32_t base = st->base, shift = st->shift;
   for (uint32_t r = lane; r < tot; r += 32) {
-    // segment w holds ranks [o_w, o_w + c_w) and starts at area + w * seg_cap
+    // segment w holds ranks [o_w, o_w + c_w)
     const uint32_t src = r >= o3 ? 3u * seg_cap + (r - o3)
                          : r >= o2 ? 2u * seg_cap + (r - o2)
                          : r >= o1 ? 1u * seg_cap + (r - o1) : r;
