@@ -66,7 +66,9 @@ typedef struct si_options {
   int query_chunk;       /* queries per launch of the chunk driver; 0 = all S in one launch.
                             Must be a multiple of 4 otherwise. */
   int key_tile;          /* keys per partition of the partition-merge: 64 or a multiple
-                            of 128 up to 1024; 0 = 512 */
+                            of 128 up to 1024; 0 = 512, or 256 / 128 / 64 when k is too
+                            large for a 512-key partition's pool in shared memory.  An
+                            explicit value whose pool does not fit gives SI_ERR_UNSUPPORTED. */
   void* workspace;       /* optional caller-owned device scratch, >= si_indexer_workspace_size() */
   size_t workspace_bytes;
   int unsorted;          /* streaming path only: 1 = leave each row's k results in an unspecified

@@ -117,7 +117,16 @@ si_status si_indexer_topk_ex(const void* q, const void* kc, const float* w, int 
     return fail(SI_ERR_INVALID_ARGUMENT, "unknown dtype %d", static_cast<int>(o.dtype));
   if (o.dtype == SI_DTYPE_FP8_E4M3 && (!o.q_scale || !o.kc_scale))
     return fail(SI_ERR_INVALID_ARGUMENT, "fp8 inputs need q_scale and kc_scale");
-  const int key_tile = o.key_tile ? o.key_tile : 512;
+  // default partition: 512 keys, halved while the pool for this k does not
+  // fit in shared memory (an explicit key_tile is taken as given)
+  int key_tile = o.key_tile;
+  if (key_tile == 0) {
+    const int fp8 = o.dtype == SI_DTYPE_FP8_E4M3;
+    int ns = 0, cap = 0;
+    size_t bytes = 0;
+    key_tile = 512;
+    while (key_tile > 64 && !stream_smem_plan(k, key_tile, fp8, &ns, &cap, &bytes)) key_tile >>= 1;
+  }
   if (!(key_tile == 64 || (key_tile % 128 == 0 && key_tile >= 128 && key_tile <= 1024)))
     return fail(SI_ERR_INVALID_ARGUMENT, "key_tile must be 64 or a multiple of 128 up to 1024 (got %d)", key_tile);
   if (o.query_chunk < 0 || (o.query_chunk % 4) != 0)

@@ -82,6 +82,41 @@ __global__ void __launch_bounds__(256) row_sort_kernel(int32_t* __restrict__ idx
   }
 }
 
+// Bitonic sort of the 32*E keys of a warp (lane l holds positions
+// [l*E, l*E+E)) into descending order.  Strides below E stay in registers;
+// larger ones exchange with lane ^ (stride / E) and keep the larger or the
+// smaller key, decided by one comparison and the direction of the stage.
+template <int E>
+__device__ __forceinline__ void warp_sort_desc(uint64_t (&v)[E], int lane) {
+#pragma unroll
+  for (int size = 2; size <= 32 * E; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      if (stride >= E) {
+        const int lm = stride / E;
+        const bool lower = (lane & lm) == 0;
+#pragma unroll
+        for (int r = 0; r < E; ++r) {
+          // descending runs where position & size == 0; the lower partner keeps the max there
+          const bool want_max = (((lane * E + r) & size) == 0) == lower;
+          const uint64_t o = topk::shfl_xor_u64(v[r], lm);
+          v[r] = ((o > v[r]) == want_max) ? o : v[r];
+        }
+      } else {
+#pragma unroll
+        for (int r = 0; r < E; ++r) {
+          if (r & stride) continue;
+          const bool desc = ((lane * E + r) & size) == 0;
+          const uint64_t a = v[r], b = v[r | stride];
+          const bool sw = (a < b) == desc;
+          v[r] = sw ? b : a;
+          v[r | stride] = sw ? a : b;
+        }
+      }
+    }
+  }
+}
+
 // Rows of up to 32*E entries, one warp per row, entirely in registers: lane
 // l holds positions [l*E, l*E+E) and the bitonic network runs in registers
 // (strides < E) and warp shuffles (strides >= E).  `vec`: k % 4 == 0 and
@@ -120,7 +155,7 @@ __global__ void __launch_bounds__(128) row_sort_warp_kernel(int32_t* __restrict_
         v[j] = i < k ? pack(sr[i], ir[i]) : 0ull;
       }
     }
-    topk::sort_regs<E>(v, lane);
+    warp_sort_desc<E>(v, lane);
     if (E >= 4 && vec) {
 #pragma unroll
       for (int j = 0; j < E; j += 4) {

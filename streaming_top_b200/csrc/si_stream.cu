@@ -232,8 +232,8 @@ struct Ctrl {
   uint64_t ring_full[RING];   // the 8 scoring warps have written the slot
   uint64_t ring_free[RING];   // the 4 managers have read the slot
   uint64_t pub[QT];           // (unit tag << 32) | threshold, published by the managers
-  topk::QState qs[QT];
-  uint32_t ring_cnt[RING][QT][4];
+  alignas(16) topk::QState qs[QT];
+  alignas(16) uint32_t ring_cnt[RING][QT][4];
   uint32_t tmem_slot;
   int abort;
 };

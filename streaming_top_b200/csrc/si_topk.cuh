@@ -14,7 +14,7 @@ namespace topk {
 constexpr int BINS = 256;
 
 // Per-query state of the running top-k (shared memory).
-struct QState {
+struct alignas(16) QState {
   uint32_t cnt;     // entries in the pool's main region
   uint32_t thr;     // candidates must have orderable score > thr
   uint32_t base;    // histogram: bin = min(255, (ord - base) >> shift)
@@ -55,33 +55,49 @@ __device__ __forceinline__ uint32_t shift_for(uint32_t span) {
 }
 
 // hist <- histogram of the orderable scores of pool[0, n).  One warp.
+// Loops over pool entries take four 32-entry chunks per step: their loads
+// are all issued before any result is used, which hides shared-memory
+// latency four times better than one chunk per step.
+constexpr int UNR = 4;
+
 __device__ __forceinline__ void hist_build(uint32_t* hist, const uint64_t* pool, int n,
                                            uint32_t base, uint32_t shift, int lane) {
   for (int i = lane; i < BINS; i += 32) hist[i] = 0u;
   __syncwarp();
-  for (int i = lane; i < n; i += 32)
-    atomicAdd(&hist[bin_of(static_cast<uint32_t>(pool[i] >> 32), base, shift)], 1u);
+  for (int i0 = 0; i0 < n; i0 += 32 * UNR) {
+    uint32_t o[UNR];
+#pragma unroll
+    for (int u = 0; u < UNR; ++u) {
+      const int i = i0 + 32 * u + lane;
+      o[u] = i < n ? static_cast<uint32_t>(pool[i] >> 32) : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < UNR; ++u)
+      if (i0 + 32 * u + lane < n) atomicAdd(&hist[bin_of(o[u], base, shift)], 1u);
+  }
   __syncwarp();
 }
 
 // The bin b at which the count of entries in bins >= b first reaches k
 // (scanning from the top), or -1 when the histogram holds fewer than k.
-// *above receives the count in bins > b.  One warp; result is warp-uniform.
+// *above receives the count in bins > b.  Lane l reads bins [8l, 8l+8) with
+// two conflict-free 16-byte loads; a suffix sum over lanes finds the lane
+// holding the crossing.  One warp; the result is warp-uniform.
 __device__ __forceinline__ int hist_find(const uint32_t* hist, uint32_t k, int lane,
                                          uint32_t* above) {
-  uint32_t c[8], sum = 0;
+  const uint4 lo = reinterpret_cast<const uint4*>(hist)[2 * lane];
+  const uint4 hi = reinterpret_cast<const uint4*>(hist)[2 * lane + 1];
+  const uint32_t c[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+  uint32_t sum = 0;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    c[i] = hist[255 - 8 * lane - i];
-    sum += c[i];
-  }
-  uint32_t incl = sum;
+  for (int i = 0; i < 8; ++i) sum += c[i];
+  uint32_t incl = sum;  // entries in bins >= 8*lane
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-    if (lane >= o) incl += v;
+    const uint32_t v = __shfl_down_sync(0xFFFFFFFFu, incl, o);
+    if (lane + o < 32) incl += v;
   }
-  const uint32_t excl = incl - sum;
+  const uint32_t excl = incl - sum;  // entries in bins >= 8*lane + 8
   const uint32_t owners = __ballot_sync(0xFFFFFFFFu, excl < k && k <= incl);
   if (!owners) return -1;
   const int owner = __ffs(owners) - 1;
@@ -90,9 +106,9 @@ __device__ __forceinline__ int hist_find(const uint32_t* hist, uint32_t k, int l
   if (lane == owner) {
     uint32_t run = excl;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 7; i >= 0; --i) {
       if (run + c[i] >= k) {
-        b = 255 - 8 * lane - i;
+        b = 8 * lane + i;
         ab = run;
         break;
       }
@@ -112,18 +128,29 @@ __device__ __forceinline__ int pool_compact(uint64_t* pool, int n, uint32_t thr,
                                             uint32_t* mx) {
   int kept = 0;
   uint32_t m = 0;
-  for (int base = 0; base < n; base += 32) {
-    const int i = base + lane;
-    const uint64_t x = i < n ? pool[i] : 0ull;
-    const uint32_t o = static_cast<uint32_t>(x >> 32);
-    const bool keep = i < n && o >= thr;
-    const uint32_t bal = __ballot_sync(0xFFFFFFFFu, keep);
-    __syncwarp();
-    if (keep) {
-      pool[kept + __popc(bal & ((1u << lane) - 1u))] = x;
-      m = o > m ? o : m;
+  const uint32_t lm = (1u << lane) - 1u;
+  for (int base = 0; base < n; base += 32 * UNR) {
+    uint64_t x[UNR];
+    bool keep[UNR];
+    uint32_t bal[UNR];
+#pragma unroll
+    for (int u = 0; u < UNR; ++u) {
+      const int i = base + 32 * u + lane;
+      x[u] = i < n ? pool[i] : 0ull;
+      keep[u] = i < n && static_cast<uint32_t>(x[u] >> 32) >= thr;
     }
-    kept += __popc(bal);
+#pragma unroll
+    for (int u = 0; u < UNR; ++u) bal[u] = __ballot_sync(0xFFFFFFFFu, keep[u]);
+    __syncwarp();  // every load of this step precedes its stores (they land at or below it)
+#pragma unroll
+    for (int u = 0; u < UNR; ++u) {
+      if (keep[u]) {
+        pool[kept + __popc(bal[u] & lm)] = x[u];
+        const uint32_t o = static_cast<uint32_t>(x[u] >> 32);
+        m = o > m ? o : m;
+      }
+      kept += __popc(bal[u]);
+    }
     __syncwarp();
   }
   *mx = warp_max_u32(m);
@@ -342,13 +369,15 @@ __device__ __forceinline__ void pool_sort(uint64_t* pool, int n, int lane) {
 __device__ __forceinline__ void merge(QState* st, uint64_t* pool, const uint64_t* area,
                                       const uint32_t* seg, int seg_cap, uint32_t* hist, int lane,
                                       int w_lo = 0, int w_hi = 4) {
-  const uint32_t c = lane >= w_lo && lane < w_hi ? seg[lane] : 0u;
-  const uint32_t c0 = __shfl_sync(0xFFFFFFFFu, c, 0), c1 = __shfl_sync(0xFFFFFFFFu, c, 1);
-  const uint32_t c2 = __shfl_sync(0xFFFFFFFFu, c, 2), c3 = __shfl_sync(0xFFFFFFFFu, c, 3);
+  // every lane reads the four counts and the state with broadcast 16-byte loads
+  const uint4 cv = *reinterpret_cast<const uint4*>(seg);
+  const uint4 sv = *reinterpret_cast<const uint4*>(st);  // cnt, thr, base, shift
+  const uint32_t c0 = w_lo <= 0 && 0 < w_hi ? cv.x : 0u, c1 = w_lo <= 1 && 1 < w_hi ? cv.y : 0u;
+  const uint32_t c2 = w_lo <= 2 && 2 < w_hi ? cv.z : 0u, c3 = w_lo <= 3 && 3 < w_hi ? cv.w : 0u;
   const uint32_t o1 = c0, o2 = c0 + c1, o3 = c0 + c1 + c2, tot = o3 + c3;
-  const uint32_t n = st->cnt;
+  const uint32_t n = sv.x;
   const bool binned = st->binned != 0;
-  const uint32_t base = st->base, shift = st->shift;
+  const uint32_t base = sv.z, shift = sv.w;
   for (uint32_t r = lane; r < tot; r += 32) {
     // segment w holds ranks [o_w, o_w + c_w)
     const uint32_t src = r >= o3 ? 3u * seg_cap + (r - o3)
@@ -383,10 +412,20 @@ __device__ inline void refresh(QState* st, uint64_t* pool, uint32_t* hist, int k
   bool binned = st->binned != 0;
   if (!binned && n >= k) {
     uint32_t mn = ~0u, mx = 0u;
-    for (int i = lane; i < n; i += 32) {
-      const uint32_t o = static_cast<uint32_t>(pool[i] >> 32);
-      mn = o < mn ? o : mn;
-      mx = o > mx ? o : mx;
+    for (int i0 = 0; i0 < n; i0 += 32 * UNR) {
+      uint32_t o[UNR];
+#pragma unroll
+      for (int u = 0; u < UNR; ++u) {
+        const int i = i0 + 32 * u + lane;
+        o[u] = i < n ? static_cast<uint32_t>(pool[i] >> 32) : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < UNR; ++u) {
+        if (i0 + 32 * u + lane < n) {
+          mn = o[u] < mn ? o[u] : mn;
+          mx = o[u] > mx ? o[u] : mx;
+        }
+      }
     }
     mn = warp_min_u32(mn);
     mx = warp_max_u32(mx);
@@ -457,11 +496,19 @@ __device__ inline void finalize(QState* st, uint64_t* pool, uint32_t* hist, int 
       // partitioning, and fall back to radix select otherwise
       int cs = 0, ce = 0;
       if (b >= 0 && nb <= 128u) {
-        for (int b0 = 0; b0 < n; b0 += 32) {
-          const int i = b0 + lane;
-          const uint32_t bx = i < n ? bin_of(static_cast<uint32_t>(pool[i] >> 32), base, shift) : 0u;
-          cs += __popc(__ballot_sync(0xFFFFFFFFu, i < n && bx > static_cast<uint32_t>(b)));
-          ce += __popc(__ballot_sync(0xFFFFFFFFu, i < n && bx == static_cast<uint32_t>(b)));
+        for (int b0 = 0; b0 < n; b0 += 32 * UNR) {
+          uint32_t bx[UNR];
+#pragma unroll
+          for (int u = 0; u < UNR; ++u) {
+            const int i = b0 + 32 * u + lane;
+            bx[u] = i < n ? bin_of(static_cast<uint32_t>(pool[i] >> 32), base, shift) : 0u;
+          }
+#pragma unroll
+          for (int u = 0; u < UNR; ++u) {
+            const bool in = b0 + 32 * u + lane < n;
+            cs += __popc(__ballot_sync(0xFFFFFFFFu, in && bx[u] > static_cast<uint32_t>(b)));
+            ce += __popc(__ballot_sync(0xFFFFFFFFu, in && bx[u] == static_cast<uint32_t>(b)));
+          }
         }
       }
       if (b >= 0 && nb <= 128u && cs == static_cast<int>(above) && ce == static_cast<int>(nb) &&
@@ -469,21 +516,28 @@ __device__ inline void finalize(QState* st, uint64_t* pool, uint32_t* hist, int 
         __syncwarp();
         uint64_t* scratch = reinterpret_cast<uint64_t*>(hist);
         int kept = 0, nbd = 0;
-        for (int b0 = 0; b0 < n; b0 += 32) {
-          const int i = b0 + lane;
-          const uint64_t x = i < n ? pool[i] : 0ull;
-          const uint32_t bx = i < n ? bin_of(static_cast<uint32_t>(x >> 32), base, shift) : 0u;
-          const bool sure = i < n && bx > static_cast<uint32_t>(b);
-          const bool edge = i < n && bx == static_cast<uint32_t>(b);
-          const uint32_t bs = __ballot_sync(0xFFFFFFFFu, sure);
-          const uint32_t be = __ballot_sync(0xFFFFFFFFu, edge);
-          const uint32_t lt = (1u << lane) - 1u;
-          const int pe = nbd + __popc(be & lt);
-          __syncwarp();
-          if (sure) pool[kept + __popc(bs & lt)] = x;
-          if (edge) scratch[pe] = x;
-          kept += __popc(bs);
-          nbd += __popc(be);
+        const uint32_t lt = (1u << lane) - 1u;
+        for (int b0 = 0; b0 < n; b0 += 32 * UNR) {
+          uint64_t x[UNR];
+          bool sure[UNR], edge[UNR];
+#pragma unroll
+          for (int u = 0; u < UNR; ++u) {
+            const int i = b0 + 32 * u + lane;
+            x[u] = i < n ? pool[i] : 0ull;
+            const uint32_t bx = i < n ? bin_of(static_cast<uint32_t>(x[u] >> 32), base, shift) : 0u;
+            sure[u] = i < n && bx > static_cast<uint32_t>(b);
+            edge[u] = i < n && bx == static_cast<uint32_t>(b);
+          }
+          __syncwarp();  // every load of this step precedes its stores (they land at or below it)
+#pragma unroll
+          for (int u = 0; u < UNR; ++u) {
+            const uint32_t bs = __ballot_sync(0xFFFFFFFFu, sure[u]);
+            const uint32_t be = __ballot_sync(0xFFFFFFFFu, edge[u]);
+            if (sure[u]) pool[kept + __popc(bs & lt)] = x[u];
+            if (edge[u]) scratch[nbd + __popc(be & lt)] = x[u];
+            kept += __popc(bs);
+            nbd += __popc(be);
+          }
           __syncwarp();
         }
         const int need = k - kept;
@@ -510,6 +564,7 @@ __device__ inline void finalize(QState* st, uint64_t* pool, uint32_t* hist, int 
     }
   }
   if (sort) pool_sort(pool, n, lane);
+#pragma unroll 4
   for (int x = lane; x < k; x += 32) {
     int32_t id = -1;
     float sc = -__int_as_float(0x7f800000);

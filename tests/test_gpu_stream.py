@@ -302,3 +302,16 @@ def test_row_sort_matches_lexicographic_order(k):
         order = np.lexsort((key_idx, -s))
         assert np.array_equal(gi[r], idx[r][order]), r
         assert np.array_equal(np.abs(gs[r]), np.abs(sc[r][order])), r
+
+
+def test_default_key_tile_falls_back_for_large_k():
+    """k=2048 with the default partition: the library picks a partition whose
+    pool fits (an explicit 512 is refused) and the result is exact."""
+    inp = _int_inputs(1, 2048, 512, seed=33)
+    q, kc, w = _dev(inp)
+    with pytest.raises(si.SIError) as e:
+        si.indexer_topk(q, kc, w, 4, 2048, key_tile=512)
+    assert e.value.status == si.SI_ERR_UNSUPPORTED
+    gi, gs = _run(inp, 4, 2048)
+    oi, osc, _ = oracle.topk(inp["q"], inp["kc"], inp["w"], 4, 2048)
+    parity.compare_exact(gi, gs, oi, osc, np.arange(2048))
