@@ -491,28 +491,13 @@ __device__ inline void finalize(QState* st, uint64_t* pool, uint32_t* hist, int 
       uint32_t above = 0;
       const int b = hist_find(hist, static_cast<uint32_t>(k), lane, &above);
       const uint32_t nb = b >= 0 ? hist[b] : 0u;
-      // the counts of the bins at and above the boundary are exact (only bins
-      // below an earlier threshold were ever zeroed); verify that before
-      // partitioning, and fall back to radix select otherwise
-      int cs = 0, ce = 0;
-      if (b >= 0 && nb <= 128u) {
-        for (int b0 = 0; b0 < n; b0 += 32 * UNR) {
-          uint32_t bx[UNR];
-#pragma unroll
-          for (int u = 0; u < UNR; ++u) {
-            const int i = b0 + 32 * u + lane;
-            bx[u] = i < n ? bin_of(static_cast<uint32_t>(pool[i] >> 32), base, shift) : 0u;
-          }
-#pragma unroll
-          for (int u = 0; u < UNR; ++u) {
-            const bool in = b0 + 32 * u + lane < n;
-            cs += __popc(__ballot_sync(0xFFFFFFFFu, in && bx[u] > static_cast<uint32_t>(b)));
-            ce += __popc(__ballot_sync(0xFFFFFFFFu, in && bx[u] == static_cast<uint32_t>(b)));
-          }
-        }
-      }
-      if (b >= 0 && nb <= 128u && cs == static_cast<int>(above) && ce == static_cast<int>(nb) &&
-          k - cs >= 0 && k - cs <= ce) {
+      // The counts of the bins at and above the boundary are exact: every pool
+      // entry is counted when it arrives or when the histogram is rebuilt from
+      // the pool, and compaction zeroes only bins below the threshold, which
+      // lies below every later boundary.  So `above` entries lie above bin b
+      // and nb in it; the k - above best of those nb complete the top k.
+      const int cs = static_cast<int>(above), ce = static_cast<int>(nb);
+      if (b >= 0 && nb <= 128u && k - cs >= 0 && k - cs <= ce) {
         __syncwarp();
         uint64_t* scratch = reinterpret_cast<uint64_t*>(hist);
         int kept = 0, nbd = 0;
@@ -534,23 +519,39 @@ __device__ inline void finalize(QState* st, uint64_t* pool, uint32_t* hist, int 
             const uint32_t bs = __ballot_sync(0xFFFFFFFFu, sure[u]);
             const uint32_t be = __ballot_sync(0xFFFFFFFFu, edge[u]);
             if (sure[u]) pool[kept + __popc(bs & lt)] = x[u];
-            if (edge[u]) scratch[nbd + __popc(be & lt)] = x[u];
+            const int pe = nbd + __popc(be & lt);
+            if (edge[u] && pe < 128) scratch[pe] = x[u];  // never past the 128-entry scratch
             kept += __popc(bs);
             nbd += __popc(be);
           }
           __syncwarp();
         }
-        const int need = k - kept;
+        nbd = min(nbd, 128);
+        const int need = max(0, min(k - kept, nbd));
         // sort the boundary entries (<= 128) and take the best `need`
-        uint64_t v[4];
+        if (nbd <= 32) {
+          uint64_t v[1] = {lane < nbd ? scratch[lane] : 0ull};
+          sort_regs<1>(v, lane);
+          if (lane < need) pool[kept + lane] = v[0];
+        } else if (nbd <= 64) {
+          uint64_t v[2];
 #pragma unroll
-        for (int r = 0; r < 4; ++r) v[r] = lane * 4 + r < nbd ? scratch[lane * 4 + r] : 0ull;
-        sort_regs<4>(v, lane);
+          for (int r = 0; r < 2; ++r) v[r] = lane * 2 + r < nbd ? scratch[lane * 2 + r] : 0ull;
+          sort_regs<2>(v, lane);
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
-          if (lane * 4 + r < need) pool[kept + lane * 4 + r] = v[r];
+          for (int r = 0; r < 2; ++r)
+            if (lane * 2 + r < need) pool[kept + lane * 2 + r] = v[r];
+        } else {
+          uint64_t v[4];
+#pragma unroll
+          for (int r = 0; r < 4; ++r) v[r] = lane * 4 + r < nbd ? scratch[lane * 4 + r] : 0ull;
+          sort_regs<4>(v, lane);
+#pragma unroll
+          for (int r = 0; r < 4; ++r)
+            if (lane * 4 + r < need) pool[kept + lane * 4 + r] = v[r];
+        }
         __syncwarp();
-        n = k;
+        n = kept + need;  // k, as the histogram's counts are exact
         done = true;
       }
       if (!done && n > k) {
