@@ -451,9 +451,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&C->ring_free[slot]);  // the slot has been read
-        if (++in_part == tpp || j == U.n_kt - 1) {
+        const bool last = j == U.n_kt - 1;
+        if (++in_part == tpp || last) {
           in_part = 0;
-          if (ok) {
+          // at the unit's end only a histogram that does not exist yet is worth
+          // building (finalize selects from it); no threshold is needed any more
+          if (ok && (!last || !st->binned)) {
             topk::refresh(st, pool, qh, k, p.cap, room, lane);
             if (lane == 0)
               *reinterpret_cast<volatile uint64_t*>(&C->pub[q]) = (static_cast<uint64_t>(i) << 32) | st->thr;

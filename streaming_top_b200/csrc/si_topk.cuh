@@ -378,14 +378,29 @@ __device__ __forceinline__ void merge(QState* st, uint64_t* pool, const uint64_t
   const uint32_t n = sv.x;
   const bool binned = st->binned != 0;
   const uint32_t base = sv.z, shift = sv.w;
-  for (uint32_t r = lane; r < tot; r += 32) {
-    // segment w holds ranks [o_w, o_w + c_w)
-    const uint32_t src = r >= o3 ? 3u * seg_cap + (r - o3)
-                         : r >= o2 ? 2u * seg_cap + (r - o2)
-                         : r >= o1 ? 1u * seg_cap + (r - o1) : r;
-    const uint64_t x = area[src];
-    pool[n + r] = x;
-    if (binned) atomicAdd(&hist[bin_of(static_cast<uint32_t>(x >> 32), base, shift)], 1u);
+  if (seg_cap == 32) {
+    // one independent copy per segment: the four loads are in flight together
+    const uint32_t cw[4] = {c0, c1, c2, c3}, ow[4] = {0u, o1, o2, o3};
+    uint64_t x[4];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) x[w] = static_cast<uint32_t>(lane) < cw[w] ? area[w * 32 + lane] : 0ull;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      if (static_cast<uint32_t>(lane) < cw[w]) {
+        pool[n + ow[w] + lane] = x[w];
+        if (binned) atomicAdd(&hist[bin_of(static_cast<uint32_t>(x[w] >> 32), base, shift)], 1u);
+      }
+    }
+  } else {
+    for (uint32_t r = lane; r < tot; r += 32) {
+      // segment w holds ranks [o_w, o_w + c_w)
+      const uint32_t src = r >= o3 ? 3u * seg_cap + (r - o3)
+                           : r >= o2 ? 2u * seg_cap + (r - o2)
+                           : r >= o1 ? 1u * seg_cap + (r - o1) : r;
+      const uint64_t x = area[src];
+      pool[n + r] = x;
+      if (binned) atomicAdd(&hist[bin_of(static_cast<uint32_t>(x >> 32), base, shift)], 1u);
+    }
   }
   __syncwarp();
   if (lane == 0) st->cnt = n + tot;
