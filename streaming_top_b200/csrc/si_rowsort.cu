@@ -82,39 +82,58 @@ __global__ void __launch_bounds__(256) row_sort_kernel(int32_t* __restrict__ idx
   }
 }
 
-// Bitonic sort of the 32*E keys of a warp (lane l holds positions
-// [l*E, l*E+E)) into descending order.  Strides below E stay in registers;
-// larger ones exchange with lane ^ (stride / E) and keep the larger or the
-// smaller key, decided by one comparison and the direction of the stage.
+// One compare-exchange stage of a bitonic network over the 32*E keys of a
+// warp (lane l holds positions [l*E, l*E+E)): partners are `stride` apart and
+// the run a position belongs to is sorted descending when
+// (position & size) == 0, ascending otherwise, flipped when !desc.  Strides
+// below E stay in registers; larger ones exchange with lane ^ (stride / E)
+// and keep the larger or the smaller key after one comparison.
 template <int E>
-__device__ __forceinline__ void warp_sort_desc(uint64_t (&v)[E], int lane) {
+__device__ __forceinline__ void bitonic_stage(uint64_t (&v)[E], int lane, int size, int stride,
+                                              bool desc) {
+  if (stride >= E) {
+    const int lm = stride / E;
+    const bool lower = (lane & lm) == 0;
 #pragma unroll
-  for (int size = 2; size <= 32 * E; size <<= 1) {
+    for (int r = 0; r < E; ++r) {
+      const bool run_desc = ((((lane * E + r) & size) == 0) == desc);
+      const bool want_max = run_desc == lower;
+      const uint64_t o = topk::shfl_xor_u64(v[r], lm);
+      v[r] = ((o > v[r]) == want_max) ? o : v[r];
+    }
+  } else {
 #pragma unroll
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      if (stride >= E) {
-        const int lm = stride / E;
-        const bool lower = (lane & lm) == 0;
-#pragma unroll
-        for (int r = 0; r < E; ++r) {
-          // descending runs where position & size == 0; the lower partner keeps the max there
-          const bool want_max = (((lane * E + r) & size) == 0) == lower;
-          const uint64_t o = topk::shfl_xor_u64(v[r], lm);
-          v[r] = ((o > v[r]) == want_max) ? o : v[r];
-        }
-      } else {
-#pragma unroll
-        for (int r = 0; r < E; ++r) {
-          if (r & stride) continue;
-          const bool desc = ((lane * E + r) & size) == 0;
-          const uint64_t a = v[r], b = v[r | stride];
-          const bool sw = (a < b) == desc;
-          v[r] = sw ? b : a;
-          v[r | stride] = sw ? a : b;
-        }
-      }
+    for (int r = 0; r < E; ++r) {
+      if (r & stride) continue;
+      const bool run_desc = ((((lane * E + r) & size) == 0) == desc);
+      const uint64_t a = v[r], b = v[r | stride];
+      const bool sw = (a < b) == run_desc;
+      v[r] = sw ? b : a;
+      v[r | stride] = sw ? a : b;
     }
   }
+}
+
+// Full bitonic sort of a warp's 32*E keys, descending (ascending if !desc).
+template <int E>
+__device__ __forceinline__ void warp_sort(uint64_t (&v)[E], int lane, bool desc) {
+#pragma unroll
+  for (int size = 2; size <= 32 * E; size <<= 1)
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) bitonic_stage<E>(v, lane, size, stride, desc);
+}
+
+// The last stages of a bitonic sort: the warp's keys form a bitonic sequence;
+// leave them sorted descending (ascending if !desc).
+template <int E>
+__device__ __forceinline__ void warp_merge(uint64_t (&v)[E], int lane, bool desc) {
+#pragma unroll
+  for (int stride = 16 * E; stride > 0; stride >>= 1) bitonic_stage<E>(v, lane, 64 * E, stride, desc);
+}
+
+template <int E>
+__device__ __forceinline__ void warp_sort_desc(uint64_t (&v)[E], int lane) {
+  warp_sort<E>(v, lane, true);
 }
 
 // Rows of up to 32*E entries, one warp per row, entirely in registers: lane
@@ -181,6 +200,78 @@ __global__ void __launch_bounds__(128) row_sort_warp_kernel(int32_t* __restrict_
   }
 }
 
+// Rows of 257..512 entries: two warps per row, 256 keys each in registers.
+// Each warp sorts its half (the first descending, the second ascending, so
+// the row is bitonic); the halves compare-exchange through shared memory for
+// the stride-256 stage; each warp then finishes its half with a descending
+// merge.  Twice the warps of the one-warp kernel at half the registers, so
+// twice the latency hiding.
+__global__ void __launch_bounds__(128) row_sort_pair_kernel(int32_t* __restrict__ idx,
+                                                            float* __restrict__ score,
+                                                            long long rows, int k, int vec) {
+  __shared__ uint64_t xbuf[2][2][256];  // [row slot of the block][half][position]
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int rs = warp >> 1, h = warp & 1;
+  const uint32_t bar_id = 1u + static_cast<uint32_t>(rs);
+  for (long long r = static_cast<long long>(blockIdx.x) * 2 + rs; r < rows;
+       r += static_cast<long long>(gridDim.x) * 2) {
+    int32_t* ir = idx + r * k;
+    float* sr = score + r * k;
+    const int p0 = h * 256 + lane * 8;
+    uint64_t v[8];
+    if (vec) {
+#pragma unroll
+      for (int j = 0; j < 8; j += 4) {
+        const int i0 = p0 + j;
+        if (i0 < k) {
+          const int4 a = *reinterpret_cast<const int4*>(ir + i0);
+          const float4 b = *reinterpret_cast<const float4*>(sr + i0);
+          v[j] = pack(b.x, a.x);
+          v[j + 1] = pack(b.y, a.y);
+          v[j + 2] = pack(b.z, a.z);
+          v[j + 3] = pack(b.w, a.w);
+        } else {
+          v[j] = v[j + 1] = v[j + 2] = v[j + 3] = 0ull;
+        }
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = p0 + j < k ? pack(sr[p0 + j], ir[p0 + j]) : 0ull;
+    }
+    warp_sort<8>(v, lane, h == 0);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) xbuf[rs][h][lane * 8 + j] = v[j];
+    asm volatile("bar.sync %0, 64;" ::"r"(bar_id) : "memory");
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint64_t o = xbuf[rs][h ^ 1][lane * 8 + j];
+      v[j] = h == 0 ? (o > v[j] ? o : v[j]) : (o < v[j] ? o : v[j]);
+    }
+    asm volatile("bar.sync %0, 64;" ::"r"(bar_id) : "memory");  // xbuf is free for the next row
+    warp_merge<8>(v, lane, true);
+    if (vec) {
+#pragma unroll
+      for (int j = 0; j < 8; j += 4) {
+        const int i0 = p0 + j;
+        if (i0 < k) {
+          int4 a;
+          float4 b;
+          unpack(v[j], &b.x, &a.x);
+          unpack(v[j + 1], &b.y, &a.y);
+          unpack(v[j + 2], &b.z, &a.z);
+          unpack(v[j + 3], &b.w, &a.w);
+          *reinterpret_cast<int4*>(ir + i0) = a;
+          *reinterpret_cast<float4*>(sr + i0) = b;
+        }
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (p0 + j < k) unpack(v[j], sr + p0 + j, ir + p0 + j);
+    }
+  }
+}
+
 template <int E>
 si_status launch_warp_sort(int32_t* idx, float* score, long long rows, int k, int n_sm, int vec,
                            cudaStream_t stream) {
@@ -209,7 +300,12 @@ si_status launch_row_sort(int32_t* idx, float* score, long long rows, int k, cud
     case 64: launch_warp_sort<2>(idx, score, rows, k, n_sm, vec, stream); break;
     case 128: launch_warp_sort<4>(idx, score, rows, k, n_sm, vec, stream); break;
     case 256: launch_warp_sort<8>(idx, score, rows, k, n_sm, vec, stream); break;
-    case 512: launch_warp_sort<16>(idx, score, rows, k, n_sm, vec, stream); break;
+    case 512: {
+      const long long blocks = (rows + 1) / 2;  // 2 rows (4 warps) per block
+      const long long grid = std::min<long long>(blocks, static_cast<long long>(n_sm) * 16);
+      row_sort_pair_kernel<<<static_cast<unsigned>(grid), 128, 0, stream>>>(idx, score, rows, k, vec);
+      break;
+    }
     default: {  // 1024, 2048: too many keys for one warp's registers
       const long long grid = std::min<long long>(rows, static_cast<long long>(n_sm) * 16);
       const size_t smem = static_cast<size_t>(np) * sizeof(uint64_t);

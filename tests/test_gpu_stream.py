@@ -279,7 +279,7 @@ def test_without_scores_rows_come_sorted():
         assert np.array_equal(gi.cpu().numpy().reshape(-1, k), oi)
 
 
-@pytest.mark.parametrize("k", [1, 7, 64, 100, 512, 1000, 2048])
+@pytest.mark.parametrize("k", [1, 7, 64, 100, 257, 301, 512, 1000, 2048])
 def test_row_sort_matches_lexicographic_order(k):
     """si_sort_topk_rows on arbitrary rows: score descending, index ascending,
     (-1, -inf) padding last; -0.0 ranks with +0.0."""
