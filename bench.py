@@ -148,7 +148,8 @@ def job_value(world: int, pairs_per_rank: int, ms_step: float) -> float:
 def oracle_sample(wl, inp, rows) -> tuple[float, int]:
     import oracle
     t0 = time.perf_counter()
-    oracle.topk(inp["q"], inp["kc"], inp["w"], wl.m, wl.k, rows=rows)
+    oracle.topk(inp["q"], inp["kc"], inp["w"], wl.m, wl.k, rows=rows, q_scale=inp.get("q_scale"),
+                kc_scale=inp.get("kc_scale"))
     dt = time.perf_counter() - t0
     pairs = int(sum(min(wl.T, (int(r) % wl.S + 1) // wl.m) for r in rows))
     return dt, pairs
@@ -158,7 +159,7 @@ def run_reference(args, wl):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    inp = synth.make_inputs(wl)
+    inp = synth.make_inputs(wl, fmt=args.fmt)
     per_step = args.ref_rows
     allrows = synth.sample_rows(per_step * (args.steps + args.warmup), wl.m * 4, wl.S, seed=wl.seed + 77)
     rng = np.random.default_rng(wl.seed)
@@ -206,10 +207,16 @@ def run_ours(args, wl):
     torch.cuda.set_device(dev)
 
     seed = rank_seed(wl, rank)
-    inp = synth.make_inputs(wl, seed=seed)
-    q = torch.from_numpy(inp["q"].view(np.int16)).view(torch.bfloat16).to(dev)
-    kc = torch.from_numpy(inp["kc"].view(np.int16)).view(torch.bfloat16).to(dev)
-    w = torch.from_numpy(inp["w"]).to(dev)
+    fp8 = args.fmt == "e4m3"
+    inp = synth.make_inputs(wl, fmt=args.fmt, seed=seed)
+
+    def host_tensor(name):
+        a = inp[name]
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if a.dtype == np.uint16 else torch.from_numpy(a)
+
+    q, kc, w = (host_tensor(n).to(dev) for n in ("q", "kc", "w"))
+    qs = torch.from_numpy(inp["q_scale"]).to(dev) if fp8 else None
+    ks = torch.from_numpy(inp["kc_scale"]).to(dev) if fp8 else None
     out_idx = torch.empty((wl.B, wl.S, wl.k), dtype=torch.int32, device=dev)
     out_score = torch.empty((wl.B, wl.S, wl.k), dtype=torch.float32, device=dev)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)  # > 126 MB L2
@@ -221,8 +228,8 @@ def run_ours(args, wl):
     # streaming kernel (rows left unsorted), then the row sort; an event
     # between them times the streaming kernel alone for the roofline
     def step(mid=None):
-        si.indexer_topk(q, kc, w, wl.m, wl.k, out_idx=out_idx, out_score=out_score, unsorted=True,
-                        stream=stream)
+        si.indexer_topk(q, kc, w, wl.m, wl.k, q_scale=qs, kc_scale=ks, out_idx=out_idx,
+                        out_score=out_score, unsorted=True, stream=stream)
         if mid is not None:
             mid.record(stream)
         si.sort_topk_rows(out_idx, out_score, stream=stream)
@@ -266,12 +273,12 @@ def run_ours(args, wl):
         ms_sort = max_over_ranks(ms_sort, dev)
 
     # end to end through the host-buffer API: H2D inputs, kernel, D2H results
-    hq = torch.from_numpy(inp["q"].view(np.int16)).view(torch.bfloat16).pin_memory()
-    hk = torch.from_numpy(inp["kc"].view(np.int16)).view(torch.bfloat16).pin_memory()
-    hw = torch.from_numpy(inp["w"]).pin_memory()
+    hq, hk, hw = (host_tensor(n).pin_memory() for n in ("q", "kc", "w"))
+    hqs = torch.from_numpy(inp["q_scale"]).pin_memory() if fp8 else None
+    hks = torch.from_numpy(inp["kc_scale"]).pin_memory() if fp8 else None
     bufs = {}
     for _ in range(max(1, args.warmup)):
-        si.indexer_topk_host(hq, hk, hw, wl.m, wl.k, device=dev, bufs=bufs)
+        si.indexer_topk_host(hq, hk, hw, wl.m, wl.k, q_scale=hqs, kc_scale=hks, device=dev, bufs=bufs)
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
     if world > 1:
@@ -279,13 +286,17 @@ def run_ours(args, wl):
     torch.cuda.synchronize(dev)
     for e0, e1 in e2e_ev:
         e0.record(stream)
-        si.indexer_topk_host(hq, hk, hw, wl.m, wl.k, device=dev, bufs=bufs, sync=False)
+        si.indexer_topk_host(hq, hk, hw, wl.m, wl.k, q_scale=hqs, kc_scale=hks, device=dev, bufs=bufs,
+                             sync=False)
         e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev) / args.steps
     if world > 1:
         e2e_ms = max_over_ranks(e2e_ms, dev)
-    h2d = hq.numel() * 2 + hk.numel() * 2 + hw.numel() * 4
+    esz = 1 if fp8 else 2
+    h2d = (hq.numel() + hk.numel()) * esz + hw.numel() * 4
+    if fp8:
+        h2d += (hqs.numel() + hks.numel()) * 4
     d2h = out_idx.numel() * 4 + out_score.numel() * 4
     del bufs
 
@@ -301,8 +312,15 @@ def run_ours(args, wl):
     value = job_value(world, P, ms_step)
     tflops = P * flop_pair / (ms_step * 1e-3) / 1e12
     kernel_tflops = P * flop_pair / (ms_kernel * 1e-3) / 1e12
-    alg_bytes = q.numel() * 2 + kc.numel() * 2 + w.numel() * 4 + out_idx.numel() * 4 + out_score.numel() * 4
-    traffic = ncu_traffic(wl.name)
+    alg_bytes = (q.numel() + kc.numel()) * esz + w.numel() * 4 + out_idx.numel() * 4 + out_score.numel() * 4
+    if fp8:
+        alg_bytes += (qs.numel() + ks.numel()) * 4
+    traffic = None if fp8 else ncu_traffic(wl.name)
+    # a contraction is measured against the peak of its own type: fp8 takes the
+    # measured bf16 matmul peak times the nominal fp8 / bf16 ratio (4.5 / 2.25)
+    peak_tc = peaks["bf16_tflops"] * (2.0 if fp8 else 1.0)
+    peak_src = (f"{peaks['source']} bf16 dense matmul, burst" +
+                (", x2 (nominal fp8 / bf16 dense ratio)" if fp8 else ""))
     cpu = None
     if world == 1 and args.cpu_seconds > 0:
         rows = synth.sample_rows(4096, wl.m * 4, wl.S, seed=wl.seed + 99)
@@ -321,21 +339,21 @@ def run_ours(args, wl):
     line = {
         "metric": METRIC, "value": value, "unit": "pairs/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(wl, world),
+        "vs_baseline": None, "dtype": args.fmt, "data": "synthetic", "config": config_dict(wl, world),
         "tflops": tflops,
         "frac_bf16_peak": tflops / peaks["bf16_tflops"],
         "frac_bf16_peak_sustained": tflops / peaks["bf16_tflops_sustained"] if peaks["bf16_tflops_sustained"] else None,
         "hbm_gbs": alg_bytes / (ms_step * 1e-3) / 1e9,
         "frac_hbm": alg_bytes / (ms_step * 1e-3) / 1e9 / peaks["hbm_gbs"],
         "peak_hbm_gb": peak_mem / 1e9,
-        "hbm_breakdown_gb": {"q": q.numel() * 2 / 1e9, "kc": kc.numel() * 2 / 1e9, "w": w.numel() * 4 / 1e9,
+        "hbm_breakdown_gb": {"q": q.numel() * esz / 1e9, "kc": kc.numel() * esz / 1e9, "w": w.numel() * 4 / 1e9,
                              "out_idx": out_idx.numel() * 4 / 1e9, "out_score": out_score.numel() * 4 / 1e9,
                              "l2_flush_buffer": flush.numel() / 1e9, "library_workspace": 0.0},
         "kernel_ms": {"stream_topk_kernel": ms_kernel, "row_sort_kernel": ms_sort},
         "roofline": {"bound": "tensor", "kernel": "stream_topk_kernel", "achieved": kernel_tflops,
-                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": kernel_tflops / peaks["bf16_tflops"],
-                     "peak_source": f"{peaks['source']} bf16 dense matmul, burst",
+                     "peak": peak_tc, "unit": "TFLOP/s",
+                     "frac": kernel_tflops / peak_tc,
+                     "peak_source": peak_src,
                      "traffic": traffic, "algorithmic_bytes": alg_bytes},
         "cpu_baseline": cpu,
         "e2e": {"value": job_value(world, P, e2e_ms), "unit": "pairs/s", "h2d_bytes_per_step": h2d,
@@ -356,6 +374,8 @@ def main() -> int:
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="v4flash", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--fmt", default="bf16", choices=["bf16", "e4m3"],
+                    help="input format: bf16 (default) or fp8 e4m3 with per-row scales")
     ap.add_argument("--ref-rows", type=int, default=32)
     args = ap.parse_args()
     wl = synth.WORKLOADS[args.workload]

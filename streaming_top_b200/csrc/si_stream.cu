@@ -521,6 +521,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         nvis[qi] = n < p.T ? n : p.T;
       }
       uint32_t thr0 = 0u, thr1 = 0u;
+      // fp8: the key scales of the next tile are fetched one tile ahead
+      const float* ks_row = OPB == 1 ? p.kc_scale + static_cast<size_t>(U.b) * p.T : nullptr;
+      float ksc_next = 1.f;
+      if (OPB == 1 && key_off < p.T) ksc_next = ks_row[key_off];
       for (int j = 0; j < U.n_kt; ++j, ++tix) {
         ok = ok && !*abort;
         if (ok && !mbar_wait_bounded(&C->t_full[acc], accph, abort, p.wait_limit_ns)) {
@@ -532,8 +536,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (ok) {
           tc_fence_after();
           const uint32_t ta = tmem + (static_cast<uint32_t>(quad * 32) << 16) + acc * NCOLS + (2 * qp) * HEADS;
-          float ksc = 1.f;
-          if (OPB == 1 && s < p.T) ksc = p.kc_scale[static_cast<size_t>(U.b) * p.T + s];
+          const float ksc = ksc_next;
+          if (OPB == 1) ksc_next = (j + 1 < U.n_kt && s + KT < p.T) ? ks_row[s + KT] : 1.f;
           {
             uint32_t x[64];
             tmem_ld32_x64(ta, x);
