@@ -96,6 +96,22 @@ SI_API si_status si_indexer_topk_ex(const void* q, const void* kc, const float* 
                              void* stream, const si_options* opt);
 
 /*
+ * Streaming indexer top-k over a range of query rows: rows row0 .. row0+R-1
+ * of every sequence, given as q [B, R, H_I, D] and w [B, R, H_I] (and for
+ * fp8, q_scale [B, R, H_I]), against all T compressed keys kc [B, T, D];
+ * results out_idx / out_score [B, R, k].  Row r is query position row0 + r
+ * for causal visibility: key s is visible iff s*m + m - 1 <= row0 + r.  A
+ * caller can so feed a long sequence's queries in chunks and hold only one
+ * chunk of q on the device (the pages' streaming of the query side); each
+ * row's result equals that of the whole-sequence call.  row0 >= 0, R >= 1,
+ * row0 + R < 2^31; everything else as si_indexer_topk_ex.  No counterpart
+ * of its own on the pages beyond that chunking of the queries.
+ */
+SI_API si_status si_indexer_topk_rows(const void* q, const void* kc, const float* w, int B, int row0,
+                                      int R, int T, int H_I, int D, int m, int k, int32_t* out_idx,
+                                      float* out_score, void* stream, const si_options* opt);
+
+/*
  * Sorts every row of a top-k result in place by (score descending, index
  * ascending): idx [rows, k] int32, score [rows, k] fp32, device memory, one
  * row per query.  Entries with index -1 and score -inf (padding) end up last.

@@ -43,6 +43,9 @@ _lib.si_indexer_topk.restype = _i
 _lib.si_indexer_topk.argtypes = _ARGS
 _lib.si_indexer_topk_ex.restype = _i
 _lib.si_indexer_topk_ex.argtypes = _ARGS + [ctypes.POINTER(Options)]
+_lib.si_indexer_topk_rows.restype = _i
+_lib.si_indexer_topk_rows.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp,
+                                      ctypes.POINTER(Options)]
 _lib.si_sort_topk_rows.restype = _i
 _lib.si_sort_topk_rows.argtypes = [_vp, _vp, ctypes.c_int64, _i, _vp]
 _lib.si_indexer_materialize.restype = _i
@@ -152,6 +155,24 @@ def indexer_topk(q, kc, w, m: int, k: int, *, q_scale=None, kc_scale=None, query
                                  out_idx.data_ptr(), out_score.data_ptr() if out_score is not None else None,
                                  _stream_ptr(stream), ctypes.byref(o))
     _check(st, "si_indexer_topk_ex")
+    return out_idx, out_score
+
+
+def indexer_topk_rows(q, kc, w, m: int, k: int, row0: int, *, q_scale=None, kc_scale=None,
+                      query_chunk: int = 0, key_tile: int = 0, out_idx=None, out_score=None,
+                      with_score: bool = True, unsorted: bool = False, stream=None):
+    """Streaming top-k for query rows row0 .. row0+R-1 (``si_indexer_topk_rows``):
+    q [B, R, H_I, D] and w [B, R, H_I] hold those rows only, kc [B, T, D] all
+    keys.  Returns (idx, score) of shape [B, R, k]."""
+    B, R, T, H, D = _shapes(q, kc, w)
+    out_idx, out_score = _outputs(B, R, k, q.device, out_idx, out_score, with_score)
+    o = _options(q, kc, q_scale, kc_scale, query_chunk, key_tile)
+    o.unsorted = int(bool(unsorted))
+    st = _lib.si_indexer_topk_rows(q.data_ptr(), kc.data_ptr(), w.data_ptr(), B, int(row0), R, T, H, D,
+                                   m, k, out_idx.data_ptr(),
+                                   out_score.data_ptr() if out_score is not None else None,
+                                   _stream_ptr(stream), ctypes.byref(o))
+    _check(st, "si_indexer_topk_rows")
     return out_idx, out_score
 
 

@@ -103,13 +103,19 @@ si_status check_common(const void* q, const void* kc, const float* w, int B, int
 
 using namespace si;
 
-extern "C" {
+namespace {
 
-si_status si_indexer_topk_ex(const void* q, const void* kc, const float* w, int B, int S, int T,
-                             int H_I, int D, int m, int k, int32_t* out_idx, float* out_score,
-                             void* stream, const si_options* opt) {
+// The streaming top-k over rows row0 .. row0+S-1 of every sequence (S rows
+// held in q, w and the outputs); row0 = 0, S = sequence length is the
+// whole-sequence call.
+si_status stream_topk_rows(const void* q, const void* kc, const float* w, int B, int row0, int S,
+                           int T, int H_I, int D, int m, int k, int32_t* out_idx, float* out_score,
+                           void* stream, const si_options* opt) {
   si_status st = check_common(q, kc, w, B, S, T, H_I, D, m, k, out_idx, out_score);
   if (st != SI_OK) return st;
+  if (row0 < 0) return fail(SI_ERR_INVALID_ARGUMENT, "row0 must be >= 0 (got %d)", row0);
+  if (static_cast<long long>(row0) + S > 0x7FFFFFFFll)
+    return fail(SI_ERR_UNSUPPORTED, "row0 + rows must fit in 31 bits");
   si_options o;
   std::memset(&o, 0, sizeof o);
   if (opt) o = *opt;
@@ -145,12 +151,29 @@ si_status si_indexer_topk_ex(const void* q, const void* kc, const float* w, int 
   cfg.wait_limit_ns = kDefaultWaitLimitNs;
   cfg.test_withhold = 0;
   cfg.unsorted = o.unsorted != 0;
+  cfg.row0 = row0;
   st = launch_stream_topk(q, kc, w, B, S, T, H_I, D, m, k, out_idx, out_score,
                           static_cast<cudaStream_t>(stream), cfg);
   if (st != SI_OK || cfg.unsorted || !out_score) return st;
   // the kernel left each row's k results in pool order: sort them now
   return launch_row_sort(out_idx, out_score, static_cast<long long>(B) * S, k,
                          static_cast<cudaStream_t>(stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+si_status si_indexer_topk_ex(const void* q, const void* kc, const float* w, int B, int S, int T,
+                             int H_I, int D, int m, int k, int32_t* out_idx, float* out_score,
+                             void* stream, const si_options* opt) {
+  return stream_topk_rows(q, kc, w, B, 0, S, T, H_I, D, m, k, out_idx, out_score, stream, opt);
+}
+
+si_status si_indexer_topk_rows(const void* q, const void* kc, const float* w, int B, int row0, int R,
+                               int T, int H_I, int D, int m, int k, int32_t* out_idx,
+                               float* out_score, void* stream, const si_options* opt) {
+  return stream_topk_rows(q, kc, w, B, row0, R, T, H_I, D, m, k, out_idx, out_score, stream, opt);
 }
 
 si_status si_sort_topk_rows(int32_t* idx, float* score, int64_t rows, int k, void* stream) {

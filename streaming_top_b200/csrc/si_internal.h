@@ -39,6 +39,7 @@ struct StreamConfig {
   uint64_t wait_limit_ns;
   int test_withhold;  // test hook: withhold one key-tile load (timeout path)
   bool unsorted;      // leave rows in pool order (no in-kernel sort either)
+  int row0 = 0;       // absolute position of the first query row held (row ranges)
 };
 
 // Sorts rows [rows, k] of (idx, score) in place by (score desc, index asc).

@@ -101,7 +101,8 @@ struct Params {
   int32_t* out_idx;       // [B,S,k]
   float* out_score;       // [B,S,k] or null
   int* err;               // device error record
-  int B, S, T, m, k;
+  int B, S, T, m, k;      // S: rows held per sequence (q, w and outputs hold S rows)
+  int row0;               // absolute position of row 0 (causal visibility uses row0 + t)
   int qt_begin, qt_end;   // query tiles (per sequence) of this launch
   int key_tile;           // partition length in keys (64 or multiple of 128)
   int cap;                // main-region entries per query pool
@@ -121,7 +122,7 @@ __device__ __forceinline__ Unit decode_unit(int u, const Params& p) {
   const int qt = p.qt_end - 1 - u / p.B;
   r.t0 = qt * QT;
   const int t_last = min(r.t0 + QT, p.S) - 1;
-  const int n = (t_last + 1) / p.m;
+  const int n = (p.row0 + t_last + 1) / p.m;
   r.n_keys = n < p.T ? n : p.T;
   r.n_kt = (r.n_keys + KT - 1) / KT;
   return r;
@@ -517,7 +518,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
       for (int qi = 0; qi < 2; ++qi) {
         const int t = U.t0 + 2 * qp + qi;
-        const int n = t < p.S ? (t + 1) / p.m : 0;
+        const int n = t < p.S ? (p.row0 + t + 1) / p.m : 0;
         nvis[qi] = n < p.T ? n : p.T;
       }
       uint32_t thr0 = 0u, thr1 = 0u;
@@ -665,6 +666,7 @@ si_status launch_stream_topk(const void* q, const void* kc, const float* w, int 
   p.err = err;
   p.B = B;
   p.S = S;
+  p.row0 = cfg.row0;
   p.T = T;
   p.m = m;
   p.k = k;

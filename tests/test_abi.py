@@ -98,3 +98,13 @@ def test_workspace_size():
 ])
 def test_row_sort_validation(idx, score, rows, k, status):
     assert si.lib().si_sort_topk_rows(idx, score, rows, k, None) == status
+
+
+def test_row_range_validation():
+    L = si.lib()
+    o = si.Options()
+    # a negative first row is refused on the host, before any device work
+    assert L.si_indexer_topk_rows(P, P, P, 1, -4, 64, 16, 64, 128, 4, 8, P, None, None,
+                                  ctypes.byref(o)) == si.SI_ERR_INVALID_ARGUMENT
+    assert L.si_indexer_topk_rows(P, P, P, 1, 0x7FFFFFF0, 64, 16, 64, 128, 4, 8, P, None, None,
+                                  ctypes.byref(o)) == si.SI_ERR_UNSUPPORTED

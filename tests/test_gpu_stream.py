@@ -315,3 +315,27 @@ def test_default_key_tile_falls_back_for_large_k():
     gi, gs = _run(inp, 4, 2048)
     oi, osc, _ = oracle.topk(inp["q"], inp["kc"], inp["w"], 4, 2048)
     parity.compare_exact(gi, gs, oi, osc, np.arange(2048))
+
+
+@pytest.mark.parametrize("B,S,T,bounds", [
+    (1, 2048, 512, [0, 512, 1100, 2048]),        # chunks, one not a multiple of 4
+    (2, 1030, 256, [0, 3, 517, 1030]),           # two sequences, tiny first chunk
+])
+def test_row_ranges_equal_the_whole_sequence(B, S, T, bounds):
+    """Rows fed in chunks through si_indexer_topk_rows give exactly the rows of
+    the whole-sequence call (integer inputs: bit for bit, also vs the oracle)."""
+    inp = _int_inputs(B, S, T, seed=41 + S)
+    q, kc, w = _dev(inp)
+    k = 96
+    gi, gs = si.indexer_topk(q, kc, w, 4, k)
+    parts_i, parts_s = [], []
+    for r0, r1 in zip(bounds[:-1], bounds[1:]):
+        ci, cs = si.indexer_topk_rows(q[:, r0:r1].contiguous(), kc, w[:, r0:r1].contiguous(), 4, k, r0)
+        parts_i.append(ci)
+        parts_s.append(cs)
+    assert si.device_status() == si.SI_OK
+    ri, rs = torch.cat(parts_i, dim=1), torch.cat(parts_s, dim=1)
+    assert torch.equal(ri, gi) and torch.equal(rs, gs)
+    oi, osc, _ = oracle.topk(inp["q"], inp["kc"], inp["w"], 4, k)
+    parity.compare_exact(ri.cpu().numpy().reshape(-1, k), rs.cpu().numpy().reshape(-1, k), oi, osc,
+                         np.arange(B * S))
