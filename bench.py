@@ -117,12 +117,23 @@ class ClockSampler:
                 "power_w_max": max(power) if power else None, "reasons": sorted(reasons)}
 
 
-def config_dict(wl, n_gpus: int) -> dict:
-    return {"workload": f"{wl.name}: B={wl.B}, S={wl.S}, m={wl.m} (T={wl.T}), H_I={wl.H}, D={wl.D}, "
-                        f"k={wl.k}, {wl.kind} inputs, seed {wl.seed}",
-            "B_per_gpu": wl.B, "S": wl.S, "T": wl.T, "H_I": wl.H, "D": wl.D, "m": wl.m, "k": wl.k,
-            "visible_pairs_per_gpu": wl.visible_pairs(), "parallelism": f"independent sequences x{n_gpus}",
-            "l2": "q (1 GiB) > L2, and L2 flushed before each timed step"}
+def config_dict(wl, n_gpus: int, shard: str = "seq", bounds=None) -> dict:
+    c = {"workload": f"{wl.name}: B={wl.B}, S={wl.S}, m={wl.m} (T={wl.T}), H_I={wl.H}, D={wl.D}, "
+                     f"k={wl.k}, {wl.kind} inputs, seed {wl.seed}",
+         "B_per_gpu": wl.B, "S": wl.S, "T": wl.T, "H_I": wl.H, "D": wl.D, "m": wl.m, "k": wl.k,
+         "visible_pairs_per_gpu": wl.visible_pairs(), "parallelism": f"independent sequences x{n_gpus}",
+         "l2": "q (1 GiB) > L2, and L2 flushed before each timed step"}
+    if shard == "rows":
+        c["parallelism"] = f"row shards x{n_gpus} of the same sequences (equal visible pairs, keys replicated)"
+        c["row_bounds"] = bounds
+        c["visible_pairs_total"] = wl.visible_pairs()
+        c["visible_pairs_per_gpu"] = wl.visible_pairs() / n_gpus
+    return c
+
+
+def shard_pairs(wl, r0: int, r1: int) -> int:
+    """Visible pairs of query rows r0 .. r1-1 over the B sequences."""
+    return wl.B * (synth.visible_pairs(r1, wl.T, wl.m) - synth.visible_pairs(r0, wl.T, wl.m))
 
 
 # ------------------------------------------------------------------ CPU oracle
@@ -173,11 +184,15 @@ def run_reference(args, wl):
             pairs.append(pr)
     tot_t, tot_p = sum(times), sum(pairs)
     value = tot_p / tot_t
+    ref_bounds = None
+    if args.shard == "rows":
+        import streaming_top_b200 as si  # the row partition only (host arithmetic)
+        ref_bounds = si.row_shards(wl.S, wl.T, wl.m, args.gpus)
     line = {
         "metric": METRIC, "value": value, "unit": "pairs/s", "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_dict(wl, args.gpus), "impl": "reference",
+        "scaling": "strong" if args.shard == "rows" else "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_dict(wl, args.gpus, args.shard, ref_bounds), "impl": "reference",
         "cpu_baseline": {"value": value, "unit": "pairs/s", "cores": 1, "kind": "oracle",
                          "sample": f"{per_step} sampled query rows per step of the {wl.name} workload "
                                    f"({tot_p // args.steps} visible pairs per step on average), "
@@ -206,9 +221,27 @@ def run_ours(args, wl):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
 
-    seed = rank_seed(wl, rank)
     fp8 = args.fmt == "e4m3"
-    inp = synth.make_inputs(wl, fmt=args.fmt, seed=seed)
+    rows_mode = args.shard == "rows"
+    if rows_mode:
+        # every rank holds the same sequences' keys and weights and only its
+        # own query rows (equal visible pairs per rank)
+        bounds = si.row_shards(wl.S, wl.T, wl.m, world)
+        r0, r1 = bounds[rank], bounds[rank + 1]
+        if r1 <= r0:
+            raise RuntimeError(f"rank {rank} has an empty row shard: {bounds}")
+        inp = synth.make_inputs(wl, fmt=args.fmt, seed=wl.seed, skip_q=True)
+        inp["w"] = np.ascontiguousarray(inp["w"][:, r0:r1])
+        qr = [synth.q_rows(wl, b, r0, r1 - r0, args.fmt, wl.seed) for b in range(wl.B)]
+        if fp8:
+            inp["q"] = np.stack([a for a, _ in qr])
+            inp["q_scale"] = np.stack([sc for _, sc in qr])
+        else:
+            inp["q"] = np.stack(qr)
+        rows_here = r1 - r0
+    else:
+        bounds, r0, rows_here = None, None, wl.S
+        inp = synth.make_inputs(wl, fmt=args.fmt, seed=rank_seed(wl, rank))
 
     def host_tensor(name):
         a = inp[name]
@@ -217,8 +250,8 @@ def run_ours(args, wl):
     q, kc, w = (host_tensor(n).to(dev) for n in ("q", "kc", "w"))
     qs = torch.from_numpy(inp["q_scale"]).to(dev) if fp8 else None
     ks = torch.from_numpy(inp["kc_scale"]).to(dev) if fp8 else None
-    out_idx = torch.empty((wl.B, wl.S, wl.k), dtype=torch.int32, device=dev)
-    out_score = torch.empty((wl.B, wl.S, wl.k), dtype=torch.float32, device=dev)
+    out_idx = torch.empty((wl.B, rows_here, wl.k), dtype=torch.int32, device=dev)
+    out_score = torch.empty((wl.B, rows_here, wl.k), dtype=torch.float32, device=dev)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)  # > 126 MB L2
     stream = torch.cuda.current_stream(dev)
     torch.cuda.synchronize(dev)
@@ -228,8 +261,12 @@ def run_ours(args, wl):
     # streaming kernel (rows left unsorted), then the row sort; an event
     # between them times the streaming kernel alone for the roofline
     def step(mid=None):
-        si.indexer_topk(q, kc, w, wl.m, wl.k, q_scale=qs, kc_scale=ks, out_idx=out_idx,
-                        out_score=out_score, unsorted=True, stream=stream)
+        if rows_mode:
+            si.indexer_topk_rows(q, kc, w, wl.m, wl.k, r0, q_scale=qs, kc_scale=ks, out_idx=out_idx,
+                                 out_score=out_score, unsorted=True, stream=stream)
+        else:
+            si.indexer_topk(q, kc, w, wl.m, wl.k, q_scale=qs, kc_scale=ks, out_idx=out_idx,
+                            out_score=out_score, unsorted=True, stream=stream)
         if mid is not None:
             mid.record(stream)
         si.sort_topk_rows(out_idx, out_score, stream=stream)
@@ -278,7 +315,8 @@ def run_ours(args, wl):
     hks = torch.from_numpy(inp["kc_scale"]).pin_memory() if fp8 else None
     bufs = {}
     for _ in range(max(1, args.warmup)):
-        si.indexer_topk_host(hq, hk, hw, wl.m, wl.k, q_scale=hqs, kc_scale=hks, device=dev, bufs=bufs)
+        si.indexer_topk_host(hq, hk, hw, wl.m, wl.k, q_scale=hqs, kc_scale=hks, device=dev, bufs=bufs,
+                             row0=r0)
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
     if world > 1:
@@ -287,7 +325,7 @@ def run_ours(args, wl):
     for e0, e1 in e2e_ev:
         e0.record(stream)
         si.indexer_topk_host(hq, hk, hw, wl.m, wl.k, q_scale=hqs, kc_scale=hks, device=dev, bufs=bufs,
-                             sync=False)
+                             sync=False, row0=r0)
         e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev) / args.steps
@@ -306,16 +344,25 @@ def run_ours(args, wl):
     if rank != 0:
         return 0
 
-    P = wl.visible_pairs()
     flop_pair = 2 * wl.H * wl.D
     peaks = load_peaks()
-    value = job_value(world, P, ms_step)
+    if rows_mode:
+        # one job (the whole sequences) over the slowest rank's time; the
+        # per-GPU figures take the average rank's share of the pairs
+        value = wl.visible_pairs() / (ms_step * 1e-3)
+        e2e_value = wl.visible_pairs() / (e2e_ms * 1e-3)
+        P = wl.visible_pairs() / world
+    else:
+        P = wl.visible_pairs()
+        value = job_value(world, P, ms_step)
+        e2e_value = job_value(world, P, e2e_ms)
     tflops = P * flop_pair / (ms_step * 1e-3) / 1e12
     kernel_tflops = P * flop_pair / (ms_kernel * 1e-3) / 1e12
     alg_bytes = (q.numel() + kc.numel()) * esz + w.numel() * 4 + out_idx.numel() * 4 + out_score.numel() * 4
     if fp8:
         alg_bytes += (qs.numel() + ks.numel()) * 4
-    traffic = None if fp8 else ncu_traffic(wl.name)
+    # the committed DRAM capture is of the whole-sequence launch
+    traffic = None if fp8 or (rows_mode and world > 1) else ncu_traffic(wl.name)
     # a contraction is measured against the peak of its own type: fp8 takes the
     # measured bf16 matmul peak times the nominal fp8 / bf16 ratio (4.5 / 2.25)
     peak_tc = peaks["bf16_tflops"] * (2.0 if fp8 else 1.0)
@@ -338,8 +385,10 @@ def run_ours(args, wl):
                          f"pairs, {t_tot:.1f} s), single-threaded C oracle, fp64, full sort"}
     line = {
         "metric": METRIC, "value": value, "unit": "pairs/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": args.fmt, "data": "synthetic", "config": config_dict(wl, world),
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "strong" if rows_mode else "weak",
+        "vs_baseline": None, "dtype": args.fmt, "data": "synthetic",
+        "config": config_dict(wl, world, args.shard, bounds),
         "tflops": tflops,
         "frac_bf16_peak": tflops / peaks["bf16_tflops"],
         "frac_bf16_peak_sustained": tflops / peaks["bf16_tflops_sustained"] if peaks["bf16_tflops_sustained"] else None,
@@ -356,7 +405,7 @@ def run_ours(args, wl):
                      "peak_source": peak_src,
                      "traffic": traffic, "algorithmic_bytes": alg_bytes},
         "cpu_baseline": cpu,
-        "e2e": {"value": job_value(world, P, e2e_ms), "unit": "pairs/s", "h2d_bytes_per_step": h2d,
+        "e2e": {"value": e2e_value, "unit": "pairs/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": 2 * args.steps,
         "clocks": clocks,
@@ -377,6 +426,9 @@ def main() -> int:
     ap.add_argument("--fmt", default="bf16", choices=["bf16", "e4m3"],
                     help="input format: bf16 (default) or fp8 e4m3 with per-row scales")
     ap.add_argument("--ref-rows", type=int, default=32)
+    ap.add_argument("--shard", default="seq", choices=["seq", "rows"],
+                    help="N>1: independent sequences per GPU (seq, weak scaling) or the same sequences' "
+                         "query rows split over the GPUs at equal visible pairs (rows, strong scaling)")
     args = ap.parse_args()
     wl = synth.WORKLOADS[args.workload]
     if args.impl == "reference":

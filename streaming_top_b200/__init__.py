@@ -232,11 +232,13 @@ def device_status(stream=None) -> int:
 
 def indexer_topk_host(q, kc, w, m: int, k: int, *, q_scale=None, kc_scale=None, device="cuda",
                       query_chunk: int = 0, key_tile: int = 0, bufs: dict | None = None,
-                      sync: bool = True):
+                      sync: bool = True, row0: int | None = None):
     """End-to-end call on HOST tensors (pinned for best speed): copies the
     inputs to the device, runs the streaming top-k, copies (idx, score) back.
     `bufs` may hold reusable device buffers from a previous call.  With
-    sync=False the copies back are only enqueued on the current stream."""
+    sync=False the copies back are only enqueued on the current stream.
+    With `row0`, q and w hold only rows row0 .. row0+R-1 of the sequences
+    (si_indexer_topk_rows)."""
     bufs = {} if bufs is None else bufs
     stream = torch.cuda.current_stream(device)
 
@@ -257,8 +259,12 @@ def indexer_topk_host(q, kc, w, m: int, k: int, *, q_scale=None, kc_scale=None, 
     if oi is None or oi.shape != (B, S, k):
         oi = bufs["out_idx"] = torch.empty((B, S, k), dtype=torch.int32, device=device)
         os_ = bufs["out_score"] = torch.empty((B, S, k), dtype=torch.float32, device=device)
-    indexer_topk(qd, kd, wd, m, k, q_scale=qs, kc_scale=ks, query_chunk=query_chunk,
-                 key_tile=key_tile, out_idx=oi, out_score=os_, stream=stream)
+    if row0 is None:
+        indexer_topk(qd, kd, wd, m, k, q_scale=qs, kc_scale=ks, query_chunk=query_chunk,
+                     key_tile=key_tile, out_idx=oi, out_score=os_, stream=stream)
+    else:
+        indexer_topk_rows(qd, kd, wd, m, k, row0, q_scale=qs, kc_scale=ks, query_chunk=query_chunk,
+                          key_tile=key_tile, out_idx=oi, out_score=os_, stream=stream)
     hi = bufs.get("h_idx")
     hs = bufs.get("h_score")
     if hi is None or hi.shape != oi.shape:
@@ -269,6 +275,43 @@ def indexer_topk_host(q, kc, w, m: int, k: int, *, q_scale=None, kc_scale=None, 
     if sync:
         stream.synchronize()
     return hi, hs
+
+
+def visible_pairs_before(t: int, T: int, m: int) -> int:
+    """Visible (query, key) pairs of query rows 0 .. t-1 of one sequence:
+    the sum over rows r < t of min(T, floor((r + 1) / m)) -- row r sees key s
+    iff s*m + m - 1 <= r and s < T.  Closed form: with x = r + 1, floor(x/m)
+    stays below T up to x = m*T - 1, and floor(x/m) summed over x = 1..N is
+    m*a*(a-1)/2 + a*(b+1) for (a, b) = divmod(N, m)."""
+    t = max(0, int(t))
+    n = min(t, m * T - 1)
+    a, b = divmod(n, m)
+    return m * a * (a - 1) // 2 + a * (b + 1) + (t - n) * T
+
+
+def row_shards(S: int, T: int, m: int, parts: int, align: int = 4) -> list[int]:
+    """Boundaries 0 = r_0 <= r_1 <= ... <= r_parts = S splitting the query
+    rows of a sequence into `parts` contiguous ranges of (nearly) equal
+    visible pairs -- the work of each range -- for row-sharding one sequence
+    over GPUs with si_indexer_topk_rows (the keys are replicated).  Inner
+    boundaries are multiples of `align` (whole 4-query work units)."""
+    if parts < 1 or S < 0:
+        raise ValueError("parts >= 1 and S >= 0 required")
+    total = visible_pairs_before(S, T, m)
+    bounds = [0]
+    for g in range(1, parts):
+        target = total * g / parts
+        lo, hi = 0, S  # smallest t with pairs_before(t) >= target
+        while lo < hi:
+            mid = (lo + hi) // 2
+            if visible_pairs_before(mid, T, m) >= target:
+                hi = mid
+            else:
+                lo = mid + 1
+        r = min(S, max(bounds[-1], int(round(lo / align)) * align))
+        bounds.append(r)
+    bounds.append(S)
+    return bounds
 
 
 def test_stream_timeout(q, kc, w, m: int, k: int, out_idx, wait_limit_ns: int, stream=None) -> int:

@@ -339,3 +339,22 @@ def test_row_ranges_equal_the_whole_sequence(B, S, T, bounds):
     oi, osc, _ = oracle.topk(inp["q"], inp["kc"], inp["w"], 4, k)
     parity.compare_exact(ri.cpu().numpy().reshape(-1, k), rs.cpu().numpy().reshape(-1, k), oi, osc,
                          np.arange(B * S))
+
+
+@pytest.mark.parametrize("parts", [2, 3, 8])
+def test_row_shards_put_together_equal_the_whole_sequence(parts):
+    """The row partition a multi-GPU run uses (equal visible pairs per part),
+    run part by part on one GPU through si_indexer_topk_rows, gives the
+    whole-sequence rows bit for bit (integer inputs)."""
+    B, S, T, k = 1, 4096, 1024, 128
+    inp = _int_inputs(B, S, T, seed=77 + parts)
+    q, kc, w = _dev(inp)
+    gi, gs = si.indexer_topk(q, kc, w, 4, k)
+    bounds = si.row_shards(S, T, 4, parts)
+    pi, ps = [], []
+    for r0, r1 in zip(bounds[:-1], bounds[1:]):
+        ci, cs = si.indexer_topk_rows(q[:, r0:r1].contiguous(), kc, w[:, r0:r1].contiguous(), 4, k, r0)
+        pi.append(ci)
+        ps.append(cs)
+    assert si.device_status() == si.SI_OK
+    assert torch.equal(torch.cat(pi, dim=1), gi) and torch.equal(torch.cat(ps, dim=1), gs)

@@ -77,3 +77,72 @@ def test_reference_arm_nonzero_rank_exits_quietly():
                        env=env, capture_output=True, text=True, timeout=120)
     assert r.returncode == 0, r.stderr
     assert r.stdout.strip() == ""
+
+
+def _rows_rank_main(rank, world, port, out_dir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import oracle
+        import streaming_top_b200 as si
+        wl = synth.WORKLOADS["tiny"]
+        S, m, k = 512, wl.m, 24
+        T = S // m
+        bounds = si.row_shards(S, T, m, world)
+        r0, r1 = bounds[rank], bounds[rank + 1]
+        # what a rank holds in the row-sharded bench: its own q rows, all keys
+        # and the weights of the same sequence (the same seed on every rank)
+        full = synth.make_inputs(wl, S=S)
+        q_r = synth.q_rows(wl, 0, r0, r1 - r0, S=S)
+        same_q = bool(np.array_equal(q_r, full["q"][0, r0:r1]))
+        oi, osc, _ = oracle.topk(full["q"], full["kc"], full["w"], m, k, rows=np.arange(r0, r1))
+        pairs = synth.visible_pairs(r1, T, m) - synth.visible_pairs(r0, T, m)
+        got = [None] * world
+        dist.all_gather_object(got, (bounds, same_q, pairs, oi, osc))
+        if rank == 0:
+            import pickle
+            with open(os.path.join(out_dir, "rows.pkl"), "wb") as f:
+                pickle.dump(got, f)
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_row_shards(tmp_path):
+    """Row sharding of one sequence: both ranks derive the same boundaries,
+    the shards tile [0, S) with equal visible pairs, each rank's q rows
+    generated alone equal that slice of the whole sequence's q, and the
+    ranks' top-k rows put together are the whole sequence's."""
+    import pickle
+
+    import oracle
+    world = 2
+    mp.start_processes(_rows_rank_main, args=(world, _free_port(), str(tmp_path)), nprocs=world,
+                       join=True, start_method="spawn")
+    got = pickle.load(open(tmp_path / "rows.pkl", "rb"))
+    bounds = got[0][0]
+    assert all(g[0] == bounds for g in got)
+    assert bounds[0] == 0 and bounds[-1] == 512 and all(a < b for a, b in zip(bounds, bounds[1:]))
+    assert all(g[1] for g in got)
+    pairs = [g[2] for g in got]
+    assert sum(pairs) == synth.visible_pairs(512, 128, 4)
+    assert max(pairs) / min(pairs) < 1.03
+    wl = synth.WORKLOADS["tiny"]
+    full = synth.make_inputs(wl, S=512)
+    ai, asc, _ = oracle.topk(full["q"], full["kc"], full["w"], 4, 24)
+    assert np.array_equal(np.concatenate([g[3] for g in got]), ai)
+    assert np.array_equal(np.concatenate([g[4] for g in got]), asc)
+
+
+def test_row_shards_balance_and_cover():
+    import streaming_top_b200 as si
+    for S, T, m in [(65536, 16384, 4), (1048576, 262144, 4), (1000, 100, 4), (513, 171, 3)]:
+        assert si.visible_pairs_before(S, T, m) == synth.visible_pairs(S, T, m)
+        for parts in (1, 2, 4, 8):
+            b = si.row_shards(S, T, m, parts)
+            assert b[0] == 0 and b[-1] == S and len(b) == parts + 1
+            assert all(x <= y for x, y in zip(b, b[1:]))
+            assert all(x % 4 == 0 for x in b[1:-1])
+            p = [si.visible_pairs_before(y, T, m) - si.visible_pairs_before(x, T, m) for x, y in zip(b, b[1:])]
+            if S >= 65536:
+                assert max(p) / min(p) < 1.001
