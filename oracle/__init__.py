@@ -49,6 +49,14 @@ def load(path: str | None = None):
     L.oracle_topk_bf16.argtypes = [vp, vp, vp] + [i64] * 7 + [vp, i64, vp, vp, vp]
     L.oracle_topk_e4m3.restype = ctypes.c_int
     L.oracle_topk_e4m3.argtypes = [vp, vp, vp, vp, vp] + [i64] * 7 + [vp, i64, vp, vp, vp]
+    L.oracle_e2m1_value.restype = ctypes.c_double
+    L.oracle_e2m1_value.argtypes = [ctypes.c_uint8]
+    L.oracle_e8m0_value.restype = ctypes.c_double
+    L.oracle_e8m0_value.argtypes = [ctypes.c_uint8]
+    L.oracle_topk_mxfp4.restype = ctypes.c_int
+    L.oracle_topk_mxfp4.argtypes = [vp, vp, vp, vp] + [i64] * 7 + [vp, i64, vp, vp, vp]
+    L.oracle_mxfp4_decode.restype = ctypes.c_int
+    L.oracle_mxfp4_decode.argtypes = [vp, vp, i64, i64, vp]
     L.oracle_scores_bf16.restype = ctypes.c_int
     L.oracle_scores_bf16.argtypes = [vp, vp, vp] + [i64] * 6 + [i64, vp]
     if path is None:
@@ -62,12 +70,16 @@ def _c(a: np.ndarray, dtype) -> np.ndarray:
     return a
 
 
-def topk(q, kc, w, m: int, k: int, rows=None, q_scale=None, kc_scale=None, lib=None):
+def topk(q, kc, w, m: int, k: int, rows=None, q_scale=None, kc_scale=None, lib=None,
+         kc_mx_scale=None):
     """Oracle top-k.
 
     q: [B,S,H,D] bf16 bits (uint16) or e4m3 codes (uint8, then q_scale
     [B,S,H] float32 and kc_scale [B,T] float32 are required); kc: [B,T,D];
-    w: [B,S,H] float32.  rows: flat row ids b*S+t (default: all rows).
+    w: [B,S,H] float32.  With kc_mx_scale ([B,T,D/32] E8M0 bytes), q is
+    bf16 and kc holds MXFP4 codes [B,T,D/2] (value d in the low nibble of
+    byte d/2 when d is even, the high nibble when odd).
+    rows: flat row ids b*S+t (default: all rows).
     Returns (idx int32 [n,k], score float32 [n,k], score64 float64 [n,k]).
     """
     L = lib or load()
@@ -81,7 +93,13 @@ def topk(q, kc, w, m: int, k: int, rows=None, q_scale=None, kc_scale=None, lib=N
     sc = np.empty((n, k), dtype=np.float32)
     sc64 = np.empty((n, k), dtype=np.float64)
     w = _c(w, np.float32)
-    if q.dtype == np.uint16:
+    if kc_mx_scale is not None:
+        q, kc, ms = _c(q, np.uint16), _c(kc, np.uint8), _c(kc_mx_scale, np.uint8)
+        assert kc.shape[2] * 2 == D and ms.shape == (B, T, D // 32), (kc.shape, ms.shape)
+        rc = L.oracle_topk_mxfp4(q.ctypes.data, kc.ctypes.data, ms.ctypes.data, w.ctypes.data, B, S, T, H, D,
+                                 m, k, rows.ctypes.data, n, idx.ctypes.data, sc.ctypes.data,
+                                 sc64.ctypes.data)
+    elif q.dtype == np.uint16:
         q, kc = _c(q, np.uint16), _c(kc, np.uint16)
         rc = L.oracle_topk_bf16(q.ctypes.data, kc.ctypes.data, w.ctypes.data, B, S, T, H, D, m, k,
                                 rows.ctypes.data, n, idx.ctypes.data, sc.ctypes.data, sc64.ctypes.data)
@@ -94,6 +112,19 @@ def topk(q, kc, w, m: int, k: int, rows=None, q_scale=None, kc_scale=None, lib=N
     if rc != 0:
         raise ValueError(f"oracle returned {rc}")
     return idx, sc, sc64
+
+
+def mxfp4_decode(codes, scales, lib=None) -> np.ndarray:
+    """MXFP4 rows (codes [..., D/2] bytes, E8M0 scales [..., D/32]) as float64 [..., D]."""
+    L = lib or load()
+    codes, scales = _c(codes, np.uint8), _c(scales, np.uint8)
+    D = codes.shape[-1] * 2
+    rows = int(np.prod(codes.shape[:-1]))
+    assert scales.shape[-1] * 32 == D and int(np.prod(scales.shape[:-1])) == rows
+    out = np.empty(codes.shape[:-1] + (D,), dtype=np.float64)
+    if L.oracle_mxfp4_decode(codes.ctypes.data, scales.ctypes.data, rows, D, out.ctypes.data) != 0:
+        raise ValueError("oracle_mxfp4_decode failed")
+    return out
 
 
 def scores(q, kc, w, m: int, row: int, lib=None) -> np.ndarray:

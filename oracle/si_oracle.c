@@ -20,8 +20,16 @@
  * sorted by (score descending, index ascending), truncated to k, padded with
  * index -1 / score -inf when n(t) < k.
  *
+ * Key formats: bf16; fp8 E4M3 with a per-row fp32 scale; and MXFP4 (the
+ * 4-bit indexer keys named by the V4.1-Flash deployment notes, "two-level
+ * sparse attention", indexer_kv_dtype): OCP Microscaling FP4 -- E2M1 codes,
+ * two per byte, with one E8M0 power-of-two scale per 32 consecutive values
+ * along D; queries stay bf16 in that format.
+ *
  * Arithmetic: every input value is widened exactly to double (bf16 -> double
- * is exact; e4m3 -> double is exact; scales and w are fp32, exact in double),
+ * is exact; e4m3 -> double is exact; an E2M1 code times its E8M0 block scale
+ * is a power-of-two multiple of a 2-bit significand, exact in double; scales
+ * and w are fp32, exact in double),
  * dot products are summed in d order, heads in h order, all in double.  The
  * reported score is the double result rounded to float.  Plain loops,
  * single-threaded, no SIMD intrinsics; qsort for the full sort.
@@ -53,6 +61,21 @@ double oracle_e4m3_value(uint8_t bits) {
   if (e == 0) v = ldexp((double)m, -9);
   else v = ldexp(1.0 + m / 8.0, e - 7);
   return sign ? -v : v;
+}
+
+/* OCP MX FP4 E2M1, a 4-bit code: bit 3 sign, bits 2-1 exponent (bias 1),
+ * bit 0 mantissa; exponent field 0 is subnormal (mantissa * 0.5).  The
+ * magnitudes are 0, 0.5, 1, 1.5, 2, 3, 4, 6; there is no infinity or NaN. */
+double oracle_e2m1_value(uint8_t code) {
+  int sign = (code >> 3) & 1, e = (code >> 1) & 3, m = code & 1;
+  double v = e == 0 ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+  return sign ? -v : v;
+}
+
+/* OCP MX E8M0 block scale: 2^(bits - 127); 0xFF is NaN. */
+double oracle_e8m0_value(uint8_t bits) {
+  if (bits == 0xFF) return NAN;
+  return ldexp(1.0, (int)bits - 127);
 }
 
 /* Number of keys visible to query t: key s is visible iff s*m+m-1 <= t. */
@@ -94,12 +117,22 @@ static int cand_cmp(const void* pa, const void* pb) {
 
 /* Widening of one query row / key row / weight row to double. */
 typedef struct {
-  int fmt; /* 0 bf16, 1 e4m3 */
+  int fmt; /* 0 bf16, 1 e4m3, 2 bf16 queries with MXFP4 keys */
   const void* q; const float* q_scale;
   const void* kc; const float* kc_scale;
   const float* w;
   int64_t B, S, T, H, D, m;
+  const uint8_t* kc_mx; /* fmt 2: E8M0 block scales [B,T,D/32] */
 } problem_t;
+
+/* Value d of MXFP4 row r: codes [rows, D/2] bytes, value d in the low
+ * nibble of byte d/2 when d is even and in the high nibble when d is odd;
+ * scales [rows, D/32], block d/32. */
+static double mxfp4_value(const uint8_t* codes, const uint8_t* scales, int64_t r, int64_t D, int64_t d) {
+  uint8_t byte = codes[r * (D / 2) + d / 2];
+  uint8_t code = (d & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 15);
+  return oracle_e2m1_value(code) * oracle_e8m0_value(scales[r * (D / 32) + d / 32]);
+}
 
 /* qrow receives the query's H x D values transposed to D x H. */
 static void widen_query(const problem_t* p, int64_t b, int64_t t, double* qrow, double* wrow) {
@@ -108,7 +141,7 @@ static void widen_query(const problem_t* p, int64_t b, int64_t t, double* qrow, 
     wrow[h] = (double)p->w[base + h];
     for (int64_t d = 0; d < p->D; ++d) {
       int64_t i = (base + h) * p->D + d;
-      if (p->fmt == 0) qrow[d * p->H + h] = oracle_bf16_value(((const uint16_t*)p->q)[i]);
+      if (p->fmt != 1) qrow[d * p->H + h] = oracle_bf16_value(((const uint16_t*)p->q)[i]);
       else qrow[d * p->H + h] = oracle_e4m3_value(((const uint8_t*)p->q)[i]) * (double)p->q_scale[base + h];
     }
   }
@@ -119,6 +152,7 @@ static void widen_key(const problem_t* p, int64_t b, int64_t s, double* krow) {
   for (int64_t d = 0; d < p->D; ++d) {
     int64_t i = r * p->D + d;
     if (p->fmt == 0) krow[d] = oracle_bf16_value(((const uint16_t*)p->kc)[i]);
+    else if (p->fmt == 2) krow[d] = mxfp4_value((const uint8_t*)p->kc, p->kc_mx, r, p->D, d);
     else krow[d] = oracle_e4m3_value(((const uint8_t*)p->kc)[i]) * (double)p->kc_scale[r];
   }
 }
@@ -174,8 +208,27 @@ static int topk_rows(const problem_t* p, int64_t k, const int64_t* rows, int64_t
 int oracle_topk_bf16(const uint16_t* q, const uint16_t* kc, const float* w, int64_t B, int64_t S,
                      int64_t T, int64_t H, int64_t D, int64_t m, int64_t k, const int64_t* rows,
                      int64_t n_rows, int32_t* out_idx, float* out_score, double* out_score64) {
-  problem_t p = {0, q, NULL, kc, NULL, w, B, S, T, H, D, m};
+  problem_t p = {0, q, NULL, kc, NULL, w, B, S, T, H, D, m, NULL};
   return topk_rows(&p, k, rows, n_rows, out_idx, out_score, out_score64);
+}
+
+/* bf16 q [B,S,H,D]; MXFP4 kc: codes [B,T,D/2] bytes and E8M0 scales
+ * [B,T,D/32] (D a multiple of 32). */
+int oracle_topk_mxfp4(const uint16_t* q, const uint8_t* kc, const uint8_t* kc_mx_scale, const float* w,
+                      int64_t B, int64_t S, int64_t T, int64_t H, int64_t D, int64_t m, int64_t k,
+                      const int64_t* rows, int64_t n_rows, int32_t* out_idx, float* out_score,
+                      double* out_score64) {
+  if (D <= 0 || D % 32 != 0) return -1;
+  problem_t p = {2, q, NULL, kc, NULL, w, B, S, T, H, D, m, kc_mx_scale};
+  return topk_rows(&p, k, rows, n_rows, out_idx, out_score, out_score64);
+}
+
+/* The MXFP4 rows [rows, D] as doubles (D a multiple of 32). */
+int oracle_mxfp4_decode(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t D, double* out) {
+  if (rows < 0 || D <= 0 || D % 32 != 0) return -1;
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t d = 0; d < D; ++d) out[r * D + d] = mxfp4_value(codes, scales, r, D, d);
+  return 0;
 }
 
 /* e4m3 q [B,S,H,D] with q_scale [B,S,H]; e4m3 kc [B,T,D] with kc_scale [B,T];
@@ -184,7 +237,7 @@ int oracle_topk_e4m3(const uint8_t* q, const float* q_scale, const uint8_t* kc,
                      const float* kc_scale, const float* w, int64_t B, int64_t S, int64_t T,
                      int64_t H, int64_t D, int64_t m, int64_t k, const int64_t* rows,
                      int64_t n_rows, int32_t* out_idx, float* out_score, double* out_score64) {
-  problem_t p = {1, q, q_scale, kc, kc_scale, w, B, S, T, H, D, m};
+  problem_t p = {1, q, q_scale, kc, kc_scale, w, B, S, T, H, D, m, NULL};
   return topk_rows(&p, k, rows, n_rows, out_idx, out_score, out_score64);
 }
 
@@ -192,7 +245,7 @@ int oracle_topk_e4m3(const uint8_t* q, const float* q_scale, const uint8_t* kc,
  * For brute-force and invariant tests on small inputs. */
 int oracle_scores_bf16(const uint16_t* q, const uint16_t* kc, const float* w, int64_t B, int64_t S,
                        int64_t T, int64_t H, int64_t D, int64_t m, int64_t row, double* out) {
-  problem_t p = {0, q, NULL, kc, NULL, w, B, S, T, H, D, m};
+  problem_t p = {0, q, NULL, kc, NULL, w, B, S, T, H, D, m, NULL};
   if (row < 0 || row >= B * S) return -1;
   double* qrow = (double*)malloc(sizeof(double) * (size_t)(H * D));
   double* wrow = (double*)malloc(sizeof(double) * (size_t)H);

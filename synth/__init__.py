@@ -220,6 +220,29 @@ WORKLOADS = {
     "million": Workload("million", 1, 1048576, 4, 64, 128, 512, 4, "planted"),
 }
 
+def quantize_mxfp4(x: np.ndarray):
+    """OCP Microscaling FP4 of float rows [..., D] (D a multiple of 32): each
+    block of 32 consecutive values gets the E8M0 scale 2^(floor(log2 amax) - 2)
+    (2 is E2M1's largest exponent; an all-zero block gets 2^0), and each value
+    / scale is rounded to nearest-even on the E2M1 grid, saturating at +-6.
+    Returns (codes [..., D/2] uint8 -- value d in the low nibble of byte d/2
+    when d is even, the high nibble when odd -- and scales [..., D/32] uint8)."""
+    import ml_dtypes
+    x = np.asarray(x, dtype=np.float32)
+    D = x.shape[-1]
+    assert D % 32 == 0
+    blk = x.reshape(x.shape[:-1] + (D // 32, 32)).astype(np.float64)
+    amax = np.abs(blk).max(axis=-1)
+    e = np.where(amax > 0, np.floor(np.log2(np.where(amax > 0, amax, 1.0))) - 2, 0).astype(np.int64)
+    e = np.clip(e, -127, 127)
+    scales = (e + 127).astype(np.uint8)
+    v = np.clip(blk / np.ldexp(1.0, e)[..., None], -6.0, 6.0).astype(np.float32)
+    codes = v.astype(ml_dtypes.float4_e2m1fn).view(np.uint8) & 0xF
+    codes = codes.reshape(x.shape[:-1] + (D,))
+    packed = (codes[..., 0::2] | (codes[..., 1::2] << 4)).astype(np.uint8)
+    return packed, scales
+
+
 PLANTED_FRAC = 0.05
 PLANTED_BOOST = 2.0
 
@@ -234,7 +257,13 @@ def make_inputs(wl: Workload, fmt: str = "bf16", S: int | None = None, B: int | 
     `S`, `B` and `seed` override the workload's (for reduced-size cases).
     `skip_q` leaves q (and q_scale) out, for callers that make it piecewise
     with q_rows().
+    fmt "mxfp4": q as for bf16; the bf16 keys quantised by quantize_mxfp4
+    (kc: codes [B, T, D/2], kc_mx_scale: E8M0 [B, T, D/32]).
     """
+    if fmt == "mxfp4":
+        res = make_inputs(wl, "bf16", S=S, B=B, seed=seed, skip_q=skip_q)
+        res["kc"], res["kc_mx_scale"] = quantize_mxfp4(bf16_bits_to_f32(res["kc"]))
+        return res
     S = wl.S if S is None else S
     B = wl.B if B is None else B
     seed = wl.seed if seed is None else seed
@@ -282,6 +311,7 @@ def q_rows(wl: Workload, b: int, t0: int, n: int, fmt: str = "bf16", seed: int |
     [n, H, D] bf16 bits, or (e4m3 codes, q_scale [n, H])."""
     S = wl.S if S is None else S
     seed = wl.seed if seed is None else seed
+    fmt = "bf16" if fmt == "mxfp4" else fmt  # queries stay bf16 with MXFP4 keys
     kind, sig = _q_kind(wl)
     row0 = (b * S + t0) * wl.H
     res = matrix_range(row0, n * wl.H, wl.D, seed, TENSOR_Q, kind, sig, fmt, out=out, scale_out=scale_out)
@@ -298,6 +328,7 @@ def make_inputs_rows(wl: Workload, rows, fmt: str = "bf16", seed: int | None = N
     seed = wl.seed if seed is None else seed
     B, S, T, H, D = wl.B, wl.S, wl.T, wl.H, wl.D
     full = make_inputs(wl, fmt=fmt, S=S, B=B, seed=seed, skip_q=True)
+    fmt = "bf16" if fmt == "mxfp4" else fmt  # queries stay bf16 with MXFP4 keys
     qdt = np.uint16 if fmt == "bf16" else np.uint8
     q = np.empty((B, S, H, D), dtype=qdt)
     qs = np.empty((B, S, H), dtype=np.float32) if fmt != "bf16" else None

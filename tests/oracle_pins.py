@@ -219,5 +219,31 @@ def fp8_matches_bf16(lib):
     assert np.array_equal(i8, ib) and np.array_equal(s8, sb)
 
 
+def mxfp4_matches_bf16(lib):
+    """MXFP4 keys (OCP Microscaling FP4) against the bf16 path on the same
+    values.  The codes are decoded here by ml_dtypes' float4_e2m1fn (a
+    library conversion, not the oracle's bit arithmetic) times 2^(scale-127)
+    per 32-value block, value d in the low nibble of byte d/2 when d is even;
+    such keys are exact in bf16, so both oracle paths must agree bit for
+    bit, and the oracle's own decode must give the same values."""
+    import ml_dtypes
+    rng = np.random.default_rng(23)
+    B, S, T, H, D, m, k = 2, 40, 10, 3, 64, 4, 6
+    codes = rng.integers(0, 16, size=(B, T, D)).astype(np.uint8)
+    scales = rng.integers(118, 136, size=(B, T, D // 32)).astype(np.uint8)
+    step = np.ldexp(1.0, scales.astype(np.int64) - 127).repeat(32, axis=-1)
+    vals = codes.view(ml_dtypes.float4_e2m1fn).astype(np.float64) * step
+    packed = (codes[..., 0::2] | (codes[..., 1::2] << 4)).astype(np.uint8)
+    kb = _bits(vals)
+    assert np.array_equal(_f(kb), vals)  # E2M1 times a power of two is bf16-exact here
+    assert np.array_equal(oracle.mxfp4_decode(packed, scales, lib=lib), vals)
+    q = _bits(rng.standard_normal((B, S, H, D)) / 8)
+    w = rng.random((B, S, H)).astype(np.float32)
+    imx, smx, _ = oracle.topk(q, packed, w, m, k, kc_mx_scale=scales, lib=lib)
+    ib, sb, _ = oracle.topk(q, kb, w, m, k, lib=lib)
+    assert np.array_equal(imx, ib) and np.array_equal(smx, sb)
+    assert np.any(imx[:, 0] > 0)  # the keys are not all tied
+
+
 ALL = [hand_cases, onehot_matmul, positive_closed, visible_closed, causal, prefix, brute_subsets,
-       invariances, batch_independent, fp8_matches_bf16]
+       invariances, batch_independent, fp8_matches_bf16, mxfp4_matches_bf16]

@@ -32,6 +32,11 @@ MUTANTS = {
     "query_transposed": ("qrow[d * p->H + h] = oracle_bf16_value", "qrow[h * p->D + d] = oracle_bf16_value"),
     "e4m3_bias8": ("else v = ldexp(1.0 + m / 8.0, e - 7);", "else v = ldexp(1.0 + m / 8.0, e - 8);"),
     "fp8_ignore_kscale": ("* (double)p->kc_scale[r];", ";"),
+    "e2m1_bias2": ("ldexp(1.0 + 0.5 * m, e - 1)", "ldexp(1.0 + 0.5 * m, e - 2)"),
+    "mx_nibbles_swapped": ("(d & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 15)",
+                           "(d & 1) ? (uint8_t)(byte & 15) : (uint8_t)(byte >> 4)"),
+    "mx_one_scale_per_row": ("scales[r * (D / 32) + d / 32]", "scales[r * (D / 32)]"),
+    "e8m0_bias126": ("return ldexp(1.0, (int)bits - 127);", "return ldexp(1.0, (int)bits - 126);"),
 }
 
 RUNNER = r"""

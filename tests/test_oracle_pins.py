@@ -36,6 +36,41 @@ def test_e4m3_widening_all_codes(oracle_lib):
     assert oracle_lib.oracle_e4m3_value(0x38) == 1.0
 
 
+def test_mxfp4_widening_all_codes(oracle_lib):
+    """E2M1 codes and E8M0 scales against ml_dtypes' OCP MX conversions."""
+    import ml_dtypes
+    codes = np.arange(16, dtype=np.uint8)
+    want = codes.view(ml_dtypes.float4_e2m1fn).astype(np.float64)
+    got = np.array([oracle_lib.oracle_e2m1_value(int(c)) for c in codes])
+    assert np.array_equal(got, want) and np.array_equal(np.signbit(got), np.signbit(want))
+    sc = np.arange(256, dtype=np.uint8)
+    want = sc.view(ml_dtypes.float8_e8m0fnu).astype(np.float64)
+    got = np.array([oracle_lib.oracle_e8m0_value(int(c)) for c in sc])
+    assert np.array_equal(np.isnan(got), np.isnan(want))
+    fin = ~np.isnan(want)
+    assert np.array_equal(got[fin], want[fin])
+    assert oracle_lib.oracle_e2m1_value(7) == 6.0 and oracle_lib.oracle_e8m0_value(127) == 1.0
+
+
+def test_mxfp4_quantiser_round_trip(oracle_lib):
+    """The input generator's MXFP4 quantiser: values already on a block's
+    grid come back unchanged through the oracle's decode, and every block
+    scale puts the block's largest magnitude in [4, 8) before saturation."""
+    rng = np.random.default_rng(5)
+    import ml_dtypes
+    codes = rng.integers(0, 16, size=(64, 128)).astype(np.uint8)
+    codes[:, ::32] = 7  # a +6 in every block fixes its scale
+    e = rng.integers(-20, 20, size=(64, 4))
+    vals = codes.view(ml_dtypes.float4_e2m1fn).astype(np.float64) * np.ldexp(1.0, e).repeat(32, axis=-1)
+    packed, scales = synth.quantize_mxfp4(vals.astype(np.float32))
+    assert np.array_equal(scales.astype(np.int64) - 127, e)
+    assert np.array_equal(oracle.mxfp4_decode(packed, scales, lib=oracle_lib), vals)
+    x = rng.standard_normal((32, 128)).astype(np.float32)
+    _, sc = synth.quantize_mxfp4(x)
+    amax = np.abs(x.reshape(32, 4, 32)).max(-1) / np.ldexp(1.0, sc.astype(np.int64) - 127)
+    assert np.all((amax >= 4) & (amax < 8))
+
+
 def test_visible_count_definition(oracle_lib):
     # key s covers tokens [s*m, s*m+m-1]; count keys whose last token <= t
     for m in (1, 2, 3, 4, 7):
