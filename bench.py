@@ -160,7 +160,7 @@ def oracle_sample(wl, inp, rows) -> tuple[float, int]:
     import oracle
     t0 = time.perf_counter()
     oracle.topk(inp["q"], inp["kc"], inp["w"], wl.m, wl.k, rows=rows, q_scale=inp.get("q_scale"),
-                kc_scale=inp.get("kc_scale"))
+                kc_scale=inp.get("kc_scale"), kc_mx_scale=inp.get("kc_mx_scale"))
     dt = time.perf_counter() - t0
     pairs = int(sum(min(wl.T, (int(r) % wl.S + 1) // wl.m) for r in rows))
     return dt, pairs
@@ -222,6 +222,7 @@ def run_ours(args, wl):
     torch.cuda.set_device(dev)
 
     fp8 = args.fmt == "e4m3"
+    mx = args.fmt == "mxfp4"  # bf16 queries, MXFP4 keys (decoded to bf16 inside the call)
     rows_mode = args.shard == "rows"
     if rows_mode:
         # every rank holds the same sequences' keys and weights and only its
@@ -250,6 +251,7 @@ def run_ours(args, wl):
     q, kc, w = (host_tensor(n).to(dev) for n in ("q", "kc", "w"))
     qs = torch.from_numpy(inp["q_scale"]).to(dev) if fp8 else None
     ks = torch.from_numpy(inp["kc_scale"]).to(dev) if fp8 else None
+    kms = torch.from_numpy(inp["kc_mx_scale"]).to(dev) if mx else None
     out_idx = torch.empty((wl.B, rows_here, wl.k), dtype=torch.int32, device=dev)
     out_score = torch.empty((wl.B, rows_here, wl.k), dtype=torch.float32, device=dev)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)  # > 126 MB L2
@@ -263,10 +265,10 @@ def run_ours(args, wl):
     def step(mid=None):
         if rows_mode:
             si.indexer_topk_rows(q, kc, w, wl.m, wl.k, r0, q_scale=qs, kc_scale=ks, out_idx=out_idx,
-                                 out_score=out_score, unsorted=True, stream=stream)
+                                 out_score=out_score, unsorted=True, stream=stream, kc_mx_scale=kms)
         else:
             si.indexer_topk(q, kc, w, wl.m, wl.k, q_scale=qs, kc_scale=ks, out_idx=out_idx,
-                            out_score=out_score, unsorted=True, stream=stream)
+                            out_score=out_score, unsorted=True, stream=stream, kc_mx_scale=kms)
         if mid is not None:
             mid.record(stream)
         si.sort_topk_rows(out_idx, out_score, stream=stream)
@@ -313,10 +315,11 @@ def run_ours(args, wl):
     hq, hk, hw = (host_tensor(n).pin_memory() for n in ("q", "kc", "w"))
     hqs = torch.from_numpy(inp["q_scale"]).pin_memory() if fp8 else None
     hks = torch.from_numpy(inp["kc_scale"]).pin_memory() if fp8 else None
+    hkms = torch.from_numpy(inp["kc_mx_scale"]).pin_memory() if mx else None
     bufs = {}
     for _ in range(max(1, args.warmup)):
         si.indexer_topk_host(hq, hk, hw, wl.m, wl.k, q_scale=hqs, kc_scale=hks, device=dev, bufs=bufs,
-                             row0=r0)
+                             row0=r0, kc_mx_scale=hkms)
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
     if world > 1:
@@ -325,16 +328,16 @@ def run_ours(args, wl):
     for e0, e1 in e2e_ev:
         e0.record(stream)
         si.indexer_topk_host(hq, hk, hw, wl.m, wl.k, q_scale=hqs, kc_scale=hks, device=dev, bufs=bufs,
-                             sync=False, row0=r0)
+                             sync=False, row0=r0, kc_mx_scale=hkms)
         e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev) / args.steps
     if world > 1:
         e2e_ms = max_over_ranks(e2e_ms, dev)
-    esz = 1 if fp8 else 2
-    h2d = (hq.numel() + hk.numel()) * esz + hw.numel() * 4
-    if fp8:
-        h2d += (hqs.numel() + hks.numel()) * 4
+    def nbytes(*ts):
+        return sum(t.numel() * t.element_size() for t in ts if t is not None)
+
+    h2d = nbytes(hq, hk, hw, hqs, hks, hkms)
     d2h = out_idx.numel() * 4 + out_score.numel() * 4
     del bufs
 
@@ -358,11 +361,9 @@ def run_ours(args, wl):
         e2e_value = job_value(world, P, e2e_ms)
     tflops = P * flop_pair / (ms_step * 1e-3) / 1e12
     kernel_tflops = P * flop_pair / (ms_kernel * 1e-3) / 1e12
-    alg_bytes = (q.numel() + kc.numel()) * esz + w.numel() * 4 + out_idx.numel() * 4 + out_score.numel() * 4
-    if fp8:
-        alg_bytes += (qs.numel() + ks.numel()) * 4
-    # the committed DRAM capture is of the whole-sequence launch
-    traffic = None if fp8 or (rows_mode and world > 1) else ncu_traffic(wl.name)
+    alg_bytes = nbytes(q, kc, w, out_idx, out_score, qs, ks, kms)
+    # the committed DRAM capture is of the whole-sequence bf16 launch
+    traffic = None if fp8 or mx or (rows_mode and world > 1) else ncu_traffic(wl.name)
     # a contraction is measured against the peak of its own type: fp8 takes the
     # measured bf16 matmul peak times the nominal fp8 / bf16 ratio (4.5 / 2.25)
     peak_tc = peaks["bf16_tflops"] * (2.0 if fp8 else 1.0)
@@ -387,17 +388,20 @@ def run_ours(args, wl):
         "metric": METRIC, "value": value, "unit": "pairs/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "strong" if rows_mode else "weak",
-        "vs_baseline": None, "dtype": args.fmt, "data": "synthetic",
-        "config": config_dict(wl, world, args.shard, bounds),
+        "vs_baseline": None, "dtype": "bf16" if mx else args.fmt, "data": "synthetic",
+        "config": dict(config_dict(wl, world, args.shard, bounds),
+                       **({"keys": "MXFP4 (E2M1 codes, E8M0 scale per 32 values), decoded to bf16 "
+                                   "inside the call"} if mx else {})),
         "tflops": tflops,
         "frac_bf16_peak": tflops / peaks["bf16_tflops"],
         "frac_bf16_peak_sustained": tflops / peaks["bf16_tflops_sustained"] if peaks["bf16_tflops_sustained"] else None,
         "hbm_gbs": alg_bytes / (ms_step * 1e-3) / 1e9,
         "frac_hbm": alg_bytes / (ms_step * 1e-3) / 1e9 / peaks["hbm_gbs"],
         "peak_hbm_gb": peak_mem / 1e9,
-        "hbm_breakdown_gb": {"q": q.numel() * esz / 1e9, "kc": kc.numel() * esz / 1e9, "w": w.numel() * 4 / 1e9,
-                             "out_idx": out_idx.numel() * 4 / 1e9, "out_score": out_score.numel() * 4 / 1e9,
-                             "l2_flush_buffer": flush.numel() / 1e9, "library_workspace": 0.0},
+        "hbm_breakdown_gb": {"q": nbytes(q, qs) / 1e9, "kc": nbytes(kc, ks, kms) / 1e9, "w": nbytes(w) / 1e9,
+                             "out_idx": nbytes(out_idx) / 1e9, "out_score": nbytes(out_score) / 1e9,
+                             "l2_flush_buffer": flush.numel() / 1e9,
+                             "library_workspace": (wl.B * wl.T * wl.D * 2 + 256) / 1e9 if mx else 0.0},
         "kernel_ms": {"stream_topk_kernel": ms_kernel, "row_sort_kernel": ms_sort},
         "roofline": {"bound": "tensor", "kernel": "stream_topk_kernel", "achieved": kernel_tflops,
                      "peak": peak_tc, "unit": "TFLOP/s",
@@ -423,8 +427,9 @@ def main() -> int:
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="v4flash", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--fmt", default="bf16", choices=["bf16", "e4m3"],
-                    help="input format: bf16 (default) or fp8 e4m3 with per-row scales")
+    ap.add_argument("--fmt", default="bf16", choices=["bf16", "e4m3", "mxfp4"],
+                    help="input format: bf16 (default), fp8 e4m3 with per-row scales, or mxfp4 keys "
+                         "(E2M1 + E8M0 per 32 values) with bf16 queries")
     ap.add_argument("--ref-rows", type=int, default=32)
     ap.add_argument("--shard", default="seq", choices=["seq", "rows"],
                     help="N>1: independent sequences per GPU (seq, weak scaling) or the same sequences' "

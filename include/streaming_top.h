@@ -54,8 +54,13 @@ typedef enum si_status {
 } si_status;
 
 typedef enum si_dtype {
-  SI_DTYPE_BF16 = 0,     /* q, kc are bf16 */
-  SI_DTYPE_FP8_E4M3 = 1  /* q, kc are OCP fp8 e4m3 codes with per-row fp32 scales */
+  SI_DTYPE_BF16 = 0,      /* q, kc are bf16 */
+  SI_DTYPE_FP8_E4M3 = 1,  /* q, kc are OCP fp8 e4m3 codes with per-row fp32 scales */
+  SI_DTYPE_MXFP4_KEYS = 2 /* q is bf16; kc is MXFP4 (the 4-bit indexer keys of the V4.1-Flash
+                             deployment notes, "two-level sparse attention"): OCP Microscaling
+                             FP4, E2M1 codes [B,T,D/2] bytes -- value d in the low nibble of byte
+                             d/2 when d is even, the high nibble when odd -- with one E8M0 scale
+                             per 32 values along D in kc_mx_scale [B,T,D/32] */
 } si_dtype;
 
 /* Options of si_indexer_topk_ex.  Zero-initialise, then set what you need. */
@@ -74,6 +79,10 @@ typedef struct si_options {
   int unsorted;          /* streaming path only: 1 = leave each row's k results in an unspecified
                             order (valid entries first, then the -1 / -inf padding) and skip the
                             row sort; 0 (default) = sorted by score descending, index ascending */
+  const uint8_t* kc_mx_scale; /* SI_DTYPE_MXFP4_KEYS only: E8M0 block scales [B,T,D/32], value
+                            2^(byte-127) (device).  The keys are decoded to bf16 (exact for scales
+                            <= 252) into B*T*D*2 bytes of scratch -- opt->workspace when given,
+                            else allocated and freed on `stream` -- then scored as bf16. */
 } si_options;
 
 /*
@@ -160,8 +169,22 @@ SI_API si_status si_indexer_materialize_noalloc(const void* q, const void* kc, c
                                                 int B, int S, int T, int H_I, int D, int m, int k,
                                                 int32_t* out_idx, float* out_score, void* stream);
 
+/*
+ * Decodes MXFP4 rows to bf16: codes [rows, D/2] bytes (value d in the low
+ * nibble of byte d/2 when d is even, the high nibble when odd), E8M0 scales
+ * [rows, D/32] (one per 32 values), out [rows, D] bf16; device pointers,
+ * caller-owned; codes and out 16-byte aligned.  D a positive multiple of 32.
+ * An E2M1 value times 2^(scale-127) is a bf16 value exactly for scales
+ * <= 252; 253 and 254 can overflow to +-inf and 255 (NaN) gives NaN.
+ * rows >= 0 (0: nothing).  Asynchronous on `stream`.  The streaming path's
+ * key decode for SI_DTYPE_MXFP4_KEYS; also a conversion for callers.
+ */
+SI_API si_status si_mxfp4_to_bf16(const void* codes, const void* scales, int64_t rows, int D, void* out,
+                                  void* stream);
+
 /* Scratch bytes a call with these arguments needs (0 if none).  materialize
- * selects the materialize path's need. */
+ * selects the materialize path's need; otherwise the streaming path's, which
+ * is B*T*D*2 (+ alignment) for SI_DTYPE_MXFP4_KEYS and 0 for the others. */
 SI_API size_t si_indexer_workspace_size(int B, int S, int T, int H_I, int D, int m, int k, int materialize,
                                  const si_options* opt);
 

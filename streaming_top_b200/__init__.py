@@ -28,14 +28,15 @@ if not os.path.exists(LIB_PATH):
 _lib = ctypes.CDLL(LIB_PATH)
 
 SI_OK, SI_ERR_INVALID_ARGUMENT, SI_ERR_UNSUPPORTED, SI_ERR_OUT_OF_MEMORY, SI_ERR_CUDA, SI_ERR_TIMEOUT = range(6)
-SI_DTYPE_BF16, SI_DTYPE_FP8_E4M3 = 0, 1
+SI_DTYPE_BF16, SI_DTYPE_FP8_E4M3, SI_DTYPE_MXFP4_KEYS = 0, 1, 2
 
 _vp, _i, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
 
 
 class Options(ctypes.Structure):
     _fields_ = [("dtype", _i), ("q_scale", _vp), ("kc_scale", _vp), ("query_chunk", _i),
-                ("key_tile", _i), ("workspace", _vp), ("workspace_bytes", _sz), ("unsorted", _i)]
+                ("key_tile", _i), ("workspace", _vp), ("workspace_bytes", _sz), ("unsorted", _i),
+                ("kc_mx_scale", _vp)]
 
 
 _ARGS = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp]
@@ -55,6 +56,8 @@ _lib.si_indexer_materialize_noalloc.argtypes = _ARGS
 NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024  # SI_NOALLOC_SCRATCH_BYTES
 _lib.si_indexer_workspace_size.restype = _sz
 _lib.si_indexer_workspace_size.argtypes = [_i] * 8 + [ctypes.POINTER(Options)]
+_lib.si_mxfp4_to_bf16.restype = _i
+_lib.si_mxfp4_to_bf16.argtypes = [_vp, _vp, ctypes.c_int64, _i, _vp, _vp]
 _lib.si_device_status.restype = _i
 _lib.si_device_status.argtypes = [_vp]
 _lib.si_status_string.restype = ctypes.c_char_p
@@ -92,11 +95,12 @@ def _stream_ptr(stream) -> int:
     return s.cuda_stream
 
 
-def _shapes(q, kc, w):
+def _shapes(q, kc, w, mxfp4: bool = False):
     if q.dim() != 4 or kc.dim() != 3 or w.dim() != 3:
-        raise ValueError("q [B,S,H,D], kc [B,T,D], w [B,S,H] expected")
+        raise ValueError("q [B,S,H,D], kc [B,T,D] (MXFP4: [B,T,D/2] codes), w [B,S,H] expected")
     B, S, H, D = q.shape
-    if kc.shape[0] != B or kc.shape[2] != D or tuple(w.shape) != (B, S, H):
+    kd = D // 2 if mxfp4 else D
+    if kc.shape[0] != B or kc.shape[2] != kd or tuple(w.shape) != (B, S, H):
         raise ValueError(f"shape mismatch q{tuple(q.shape)} kc{tuple(kc.shape)} w{tuple(w.shape)}")
     for name, t in (("q", q), ("kc", kc), ("w", w)):
         if not t.is_cuda or not t.is_contiguous():
@@ -114,11 +118,21 @@ def _outputs(B, S, k, device, out_idx, out_score, with_score):
     return out_idx, out_score
 
 
-def _options(q, kc, q_scale, kc_scale, query_chunk, key_tile, workspace=None):
+def _options(q, kc, q_scale, kc_scale, query_chunk, key_tile, workspace=None, kc_mx_scale=None):
     o = Options()
-    if kc.element_size() != q.element_size():
+    if kc_mx_scale is not None:
+        B, _, _, D = q.shape
+        shape = (B, kc.shape[1], D // 32)
+        if q.dtype != torch.bfloat16 or kc.dtype != torch.uint8 or kc.shape[2] * 2 != D:
+            raise ValueError("MXFP4 keys: q bfloat16 [B,S,H,D] and kc uint8 codes [B,T,D/2] expected")
+        if (kc_mx_scale.dtype != torch.uint8 or tuple(kc_mx_scale.shape) != shape or not kc_mx_scale.is_cuda
+                or not kc_mx_scale.is_contiguous()):
+            raise ValueError(f"kc_mx_scale must be a contiguous uint8 CUDA tensor of shape {shape}")
+        o.dtype = SI_DTYPE_MXFP4_KEYS
+        o.kc_mx_scale = kc_mx_scale.data_ptr()
+    elif kc.element_size() != q.element_size():
         raise ValueError(f"q ({q.dtype}) and kc ({kc.dtype}) must have the same element type")
-    if q.dtype == torch.bfloat16:
+    elif q.dtype == torch.bfloat16:
         o.dtype = SI_DTYPE_BF16
     elif q.dtype in (torch.uint8, torch.float8_e4m3fn):
         if q_scale is None or kc_scale is None:
@@ -143,13 +157,14 @@ def _options(q, kc, q_scale, kc_scale, query_chunk, key_tile, workspace=None):
 
 def indexer_topk(q, kc, w, m: int, k: int, *, q_scale=None, kc_scale=None, query_chunk: int = 0,
                  key_tile: int = 0, out_idx=None, out_score=None, with_score: bool = True,
-                 unsorted: bool = False, stream=None):
+                 unsorted: bool = False, stream=None, kc_mx_scale=None, workspace=None):
     """Streaming indexer top-k (``si_indexer_topk_ex``).  Returns (idx, score).
     With unsorted=True each row's results come in an unspecified order (valid
-    entries first) and the row sort is skipped."""
-    B, S, T, H, D = _shapes(q, kc, w)
+    entries first) and the row sort is skipped.  With kc_mx_scale (uint8
+    [B,T,D/32] E8M0), kc holds MXFP4 codes [B,T,D/2] (uint8) and q is bf16."""
+    B, S, T, H, D = _shapes(q, kc, w, kc_mx_scale is not None)
     out_idx, out_score = _outputs(B, S, k, q.device, out_idx, out_score, with_score)
-    o = _options(q, kc, q_scale, kc_scale, query_chunk, key_tile)
+    o = _options(q, kc, q_scale, kc_scale, query_chunk, key_tile, workspace, kc_mx_scale)
     o.unsorted = int(bool(unsorted))
     st = _lib.si_indexer_topk_ex(q.data_ptr(), kc.data_ptr(), w.data_ptr(), B, S, T, H, D, m, k,
                                  out_idx.data_ptr(), out_score.data_ptr() if out_score is not None else None,
@@ -160,13 +175,14 @@ def indexer_topk(q, kc, w, m: int, k: int, *, q_scale=None, kc_scale=None, query
 
 def indexer_topk_rows(q, kc, w, m: int, k: int, row0: int, *, q_scale=None, kc_scale=None,
                       query_chunk: int = 0, key_tile: int = 0, out_idx=None, out_score=None,
-                      with_score: bool = True, unsorted: bool = False, stream=None):
+                      with_score: bool = True, unsorted: bool = False, stream=None, kc_mx_scale=None,
+                      workspace=None):
     """Streaming top-k for query rows row0 .. row0+R-1 (``si_indexer_topk_rows``):
     q [B, R, H_I, D] and w [B, R, H_I] hold those rows only, kc [B, T, D] all
     keys.  Returns (idx, score) of shape [B, R, k]."""
-    B, R, T, H, D = _shapes(q, kc, w)
+    B, R, T, H, D = _shapes(q, kc, w, kc_mx_scale is not None)
     out_idx, out_score = _outputs(B, R, k, q.device, out_idx, out_score, with_score)
-    o = _options(q, kc, q_scale, kc_scale, query_chunk, key_tile)
+    o = _options(q, kc, q_scale, kc_scale, query_chunk, key_tile, workspace, kc_mx_scale)
     o.unsorted = int(bool(unsorted))
     st = _lib.si_indexer_topk_rows(q.data_ptr(), kc.data_ptr(), w.data_ptr(), B, int(row0), R, T, H, D,
                                    m, k, out_idx.data_ptr(),
@@ -174,6 +190,25 @@ def indexer_topk_rows(q, kc, w, m: int, k: int, row0: int, *, q_scale=None, kc_s
                                    _stream_ptr(stream), ctypes.byref(o))
     _check(st, "si_indexer_topk_rows")
     return out_idx, out_score
+
+
+def mxfp4_to_bf16(codes, scales, out=None, stream=None):
+    """Decode MXFP4 rows (``si_mxfp4_to_bf16``): codes uint8 [..., D/2], E8M0
+    scales uint8 [..., D/32]; returns bf16 [..., D]."""
+    if codes.dtype != torch.uint8 or scales.dtype != torch.uint8:
+        raise ValueError("codes and scales must be uint8")
+    D = codes.shape[-1] * 2
+    if scales.shape[:-1] != codes.shape[:-1] or scales.shape[-1] * 32 != D:
+        raise ValueError(f"scales {tuple(scales.shape)} do not match codes {tuple(codes.shape)}")
+    for name, t in (("codes", codes), ("scales", scales)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if out is None:
+        out = torch.empty(codes.shape[:-1] + (D,), dtype=torch.bfloat16, device=codes.device)
+    rows = codes.numel() // (D // 2) if D else 0
+    _check(_lib.si_mxfp4_to_bf16(codes.data_ptr(), scales.data_ptr(), rows, D, out.data_ptr(),
+                                 _stream_ptr(stream)), "si_mxfp4_to_bf16")
+    return out
 
 
 def sort_topk_rows(idx, score, stream=None):
@@ -232,7 +267,7 @@ def device_status(stream=None) -> int:
 
 def indexer_topk_host(q, kc, w, m: int, k: int, *, q_scale=None, kc_scale=None, device="cuda",
                       query_chunk: int = 0, key_tile: int = 0, bufs: dict | None = None,
-                      sync: bool = True, row0: int | None = None):
+                      sync: bool = True, row0: int | None = None, kc_mx_scale=None):
     """End-to-end call on HOST tensors (pinned for best speed): copies the
     inputs to the device, runs the streaming top-k, copies (idx, score) back.
     `bufs` may hold reusable device buffers from a previous call.  With
@@ -253,6 +288,7 @@ def indexer_topk_host(q, kc, w, m: int, k: int, *, q_scale=None, kc_scale=None, 
     qd, kd, wd = dev("q", q), dev("kc", kc), dev("w", w)
     qs = dev("q_scale", q_scale) if q_scale is not None else None
     ks = dev("kc_scale", kc_scale) if kc_scale is not None else None
+    kms = dev("kc_mx_scale", kc_mx_scale) if kc_mx_scale is not None else None
     B, S = q.shape[0], q.shape[1]
     oi = bufs.get("out_idx")
     os_ = bufs.get("out_score")
@@ -261,10 +297,10 @@ def indexer_topk_host(q, kc, w, m: int, k: int, *, q_scale=None, kc_scale=None, 
         os_ = bufs["out_score"] = torch.empty((B, S, k), dtype=torch.float32, device=device)
     if row0 is None:
         indexer_topk(qd, kd, wd, m, k, q_scale=qs, kc_scale=ks, query_chunk=query_chunk,
-                     key_tile=key_tile, out_idx=oi, out_score=os_, stream=stream)
+                     key_tile=key_tile, out_idx=oi, out_score=os_, stream=stream, kc_mx_scale=kms)
     else:
         indexer_topk_rows(qd, kd, wd, m, k, row0, q_scale=qs, kc_scale=ks, query_chunk=query_chunk,
-                          key_tile=key_tile, out_idx=oi, out_score=os_, stream=stream)
+                          key_tile=key_tile, out_idx=oi, out_score=os_, stream=stream, kc_mx_scale=kms)
     hi = bufs.get("h_idx")
     hs = bufs.get("h_score")
     if hi is None or hi.shape != oi.shape:

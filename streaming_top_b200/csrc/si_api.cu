@@ -105,6 +105,11 @@ using namespace si;
 
 namespace {
 
+// Scratch for MXFP4 keys decoded to bf16: [B, T, D] bf16 plus alignment slack.
+size_t mxfp4_key_bytes(int B, int T, int D) {
+  return static_cast<size_t>(B) * T * D * 2 + 256;
+}
+
 // The streaming top-k over rows row0 .. row0+S-1 of every sequence (S rows
 // held in q, w and the outputs); row0 = 0, S = sequence length is the
 // whole-sequence call.
@@ -119,10 +124,15 @@ si_status stream_topk_rows(const void* q, const void* kc, const float* w, int B,
   si_options o;
   std::memset(&o, 0, sizeof o);
   if (opt) o = *opt;
-  if (o.dtype != SI_DTYPE_BF16 && o.dtype != SI_DTYPE_FP8_E4M3)
+  if (o.dtype != SI_DTYPE_BF16 && o.dtype != SI_DTYPE_FP8_E4M3 && o.dtype != SI_DTYPE_MXFP4_KEYS)
     return fail(SI_ERR_INVALID_ARGUMENT, "unknown dtype %d", static_cast<int>(o.dtype));
   if (o.dtype == SI_DTYPE_FP8_E4M3 && (!o.q_scale || !o.kc_scale))
     return fail(SI_ERR_INVALID_ARGUMENT, "fp8 inputs need q_scale and kc_scale");
+  const bool mx = o.dtype == SI_DTYPE_MXFP4_KEYS;
+  if (mx && !o.kc_mx_scale) return fail(SI_ERR_INVALID_ARGUMENT, "MXFP4 keys need kc_mx_scale");
+  if (mx && o.workspace && (o.workspace_bytes < mxfp4_key_bytes(B, T, D)))
+    return fail(SI_ERR_INVALID_ARGUMENT, "workspace of %zu bytes < %zu needed for the decoded keys",
+                o.workspace_bytes, mxfp4_key_bytes(B, T, D));
   // default partition: 512 keys, halved while the pool for this k does not
   // fit in shared memory (an explicit key_tile is taken as given)
   int key_tile = o.key_tile;
@@ -152,12 +162,34 @@ si_status stream_topk_rows(const void* q, const void* kc, const float* w, int B,
   cfg.test_withhold = 0;
   cfg.unsorted = o.unsorted != 0;
   cfg.row0 = row0;
-  st = launch_stream_topk(q, kc, w, B, S, T, H_I, D, m, k, out_idx, out_score,
-                          static_cast<cudaStream_t>(stream), cfg);
-  if (st != SI_OK || cfg.unsorted || !out_score) return st;
-  // the kernel left each row's k results in pool order: sort them now
-  return launch_row_sort(out_idx, out_score, static_cast<long long>(B) * S, k,
-                         static_cast<cudaStream_t>(stream));
+  const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  // MXFP4 keys: decode them to bf16 scratch first (exact), then score as bf16
+  void* kraw = nullptr;  // the allocation, when the library made it
+  if (mx) {
+    const size_t need = mxfp4_key_bytes(B, T, D);
+    void* base = o.workspace;
+    if (!base) {
+      cudaError_t e = cudaMallocAsync(&kraw, need, cs);
+      if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(SI_ERR_OUT_OF_MEMORY, "cudaMallocAsync(%zu) for the decoded keys: %s", need,
+                    cudaGetErrorString(e));
+      }
+      base = kraw;
+    }
+    void* kdec = reinterpret_cast<void*>((reinterpret_cast<uintptr_t>(base) + 255) & ~static_cast<uintptr_t>(255));
+    st = launch_mxfp4_to_bf16(kc, o.kc_mx_scale, static_cast<long long>(B) * T, D, kdec, cs);
+    kc = kdec;
+  }
+  if (st == SI_OK) st = launch_stream_topk(q, kc, w, B, S, T, H_I, D, m, k, out_idx, out_score, cs, cfg);
+  // the kernel leaves each row's k results in pool order: sort them now
+  if (st == SI_OK && !cfg.unsorted && out_score)
+    st = launch_row_sort(out_idx, out_score, static_cast<long long>(B) * S, k, cs);
+  if (kraw) {
+    const cudaError_t e = cudaFreeAsync(kraw, cs);
+    if (e != cudaSuccess && st == SI_OK) st = cuda_fail(e, "cudaFreeAsync");
+  }
+  return st;
 }
 
 }  // namespace
@@ -228,12 +260,23 @@ si_status si_indexer_materialize(const void* q, const void* kc, const float* w, 
 
 size_t si_indexer_workspace_size(int B, int S, int T, int H_I, int D, int m, int k, int materialize,
                                  const si_options* opt) {
-  (void)D;
   (void)m;
   (void)k;
-  (void)opt;
-  if (B < 1 || S < 1 || T < 1 || H_I < 1) return 0;
-  return materialize ? materialize_workspace_bytes(B, S, T, H_I) : 0;
+  if (B < 1 || S < 1 || T < 1 || H_I < 1 || D < 1) return 0;
+  if (materialize) return materialize_workspace_bytes(B, S, T, H_I);
+  return opt && opt->dtype == SI_DTYPE_MXFP4_KEYS ? mxfp4_key_bytes(B, T, D) : 0;
+}
+
+si_status si_mxfp4_to_bf16(const void* codes, const void* scales, int64_t rows, int D, void* out,
+                           void* stream) {
+  if (rows < 0) return fail(SI_ERR_INVALID_ARGUMENT, "rows must be >= 0 (got %lld)", static_cast<long long>(rows));
+  if (D < 32 || D % 32 != 0) return fail(SI_ERR_INVALID_ARGUMENT, "D must be a positive multiple of 32 (got %d)", D);
+  if (rows == 0) return SI_OK;
+  if (!codes || !scales || !out) return fail(SI_ERR_INVALID_ARGUMENT, "codes, scales and out must be non-null");
+  if (!aligned(codes, 16) || !aligned(out, 16))
+    return fail(SI_ERR_INVALID_ARGUMENT, "codes and out must be 16-byte aligned");
+  return launch_mxfp4_to_bf16(codes, scales, static_cast<long long>(rows), D, out,
+                              static_cast<cudaStream_t>(stream));
 }
 
 si_status si_device_status(void* stream) {
@@ -267,6 +310,6 @@ const char* si_status_string(si_status s) {
 
 const char* si_last_error(void) { return g_last_error; }
 
-int si_version(void) { return 200; }
+int si_version(void) { return 300; }
 
 }  // extern "C"

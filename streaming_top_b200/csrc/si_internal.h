@@ -42,6 +42,10 @@ struct StreamConfig {
   int row0 = 0;       // absolute position of the first query row held (row ranges)
 };
 
+// Decodes MXFP4 rows (codes [rows, D/2], E8M0 scales [rows, D/32]) to bf16 [rows, D].
+si_status launch_mxfp4_to_bf16(const void* codes, const void* scales, long long rows, int D, void* out,
+                               cudaStream_t stream);
+
 // Sorts rows [rows, k] of (idx, score) in place by (score desc, index asc).
 si_status launch_row_sort(int32_t* idx, float* score, long long rows, int k, cudaStream_t stream);
 

@@ -43,7 +43,8 @@ def _worker(args):
     else:
         inp = synth.make_inputs(wl, fmt=fmt, **overrides)
     idx, sc, sc64 = oracle.topk(inp["q"], inp["kc"], inp["w"], wl.m, k, rows=rows,
-                                q_scale=inp.get("q_scale"), kc_scale=inp.get("kc_scale"))
+                                q_scale=inp.get("q_scale"), kc_scale=inp.get("kc_scale"),
+                                kc_mx_scale=inp.get("kc_mx_scale"))
     return idx, sc, sc64
 
 
@@ -59,7 +60,8 @@ def oracle_rows(wl_name: str, rows: np.ndarray, k: int, fmt: str = "bf16", overr
     wl = synth.WORKLOADS[wl_name]
     if inputs is not None:
         return oracle.topk(inputs["q"], inputs["kc"], inputs["w"], wl.m, k, rows=rows,
-                           q_scale=inputs.get("q_scale"), kc_scale=inputs.get("kc_scale"))
+                           q_scale=inputs.get("q_scale"), kc_scale=inputs.get("kc_scale"),
+                           kc_mx_scale=inputs.get("kc_mx_scale"))
     procs = procs or max(1, min(32, (os.cpu_count() or 2)))
     # interleave rows so every worker gets a similar mix of short and long rows
     parts = [rows[i::procs] for i in range(procs) if len(rows[i::procs])]

@@ -6,6 +6,7 @@ import os
 import re
 
 import pytest
+import torch
 
 import streaming_top_b200 as si
 
@@ -108,3 +109,51 @@ def test_row_range_validation():
                                   ctypes.byref(o)) == si.SI_ERR_INVALID_ARGUMENT
     assert L.si_indexer_topk_rows(P, P, P, 1, 0x7FFFFFF0, 64, 16, 64, 128, 4, 8, P, None, None,
                                   ctypes.byref(o)) == si.SI_ERR_UNSUPPORTED
+
+
+def test_mxfp4_validation():
+    L = si.lib()
+    o = si.Options()
+    o.dtype = si.SI_DTYPE_MXFP4_KEYS
+    args = (P, P, P, 1, 64, 16, 64, 128, 4, 8, P, None, None, ctypes.byref(o))
+    assert L.si_indexer_topk_ex(*args) == si.SI_ERR_INVALID_ARGUMENT  # no block scales
+    o.kc_mx_scale = P
+    o.workspace, o.workspace_bytes = P, 64  # too small for the decoded keys
+    assert L.si_indexer_topk_ex(*args) == si.SI_ERR_INVALID_ARGUMENT
+    o.workspace, o.workspace_bytes = None, 0
+    assert L.si_indexer_workspace_size(2, 64, 16, 64, 128, 4, 8, 0, ctypes.byref(o)) == 2 * 16 * 128 * 2 + 256
+    o.dtype = si.SI_DTYPE_BF16
+    assert L.si_indexer_workspace_size(2, 64, 16, 64, 128, 4, 8, 0, ctypes.byref(o)) == 0
+    assert L.si_mxfp4_to_bf16(P, P, 4, 48, P, None) == si.SI_ERR_INVALID_ARGUMENT  # D % 32
+    assert L.si_mxfp4_to_bf16(P, P, -1, 128, P, None) == si.SI_ERR_INVALID_ARGUMENT
+    assert L.si_mxfp4_to_bf16(P + 8, P, 4, 128, P, None) == si.SI_ERR_INVALID_ARGUMENT  # alignment
+    assert L.si_mxfp4_to_bf16(P, P, 0, 128, P, None) == si.SI_OK  # nothing to do
+
+
+def test_mxfp4_options_keep_their_dtype():
+    """The binding's option marshalling for MXFP4 keys (CPU tensors stand in
+    for device ones: only shapes, dtypes and pointers are read)."""
+    q = torch.zeros((1, 8, 64, 128), dtype=torch.bfloat16)
+    kc = torch.zeros((1, 2, 64), dtype=torch.uint8)
+    ms = torch.zeros((1, 2, 4), dtype=torch.uint8)
+    o = si._options(q, kc, None, None, 0, 0, kc_mx_scale=_Cuda(ms))
+    assert o.dtype == si.SI_DTYPE_MXFP4_KEYS and o.kc_mx_scale == ms.data_ptr()
+    o = si._options(q, torch.zeros((1, 2, 128), dtype=torch.bfloat16), None, None, 0, 0)
+    assert o.dtype == si.SI_DTYPE_BF16 and not o.kc_mx_scale
+    with pytest.raises(ValueError):
+        si._options(q, torch.zeros((1, 2, 128), dtype=torch.uint8), None, None, 0, 0, kc_mx_scale=_Cuda(ms))
+
+
+class _Cuda:
+    """A CPU tensor that reports itself as a CUDA one (shape checks only)."""
+
+    def __init__(self, t):
+        self._t = t
+        self.is_cuda = True
+        self.dtype, self.shape = t.dtype, t.shape
+
+    def is_contiguous(self):
+        return True
+
+    def data_ptr(self):
+        return self._t.data_ptr()
