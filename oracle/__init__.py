@@ -57,6 +57,10 @@ def load(path: str | None = None):
     L.oracle_topk_mxfp4.argtypes = [vp, vp, vp, vp] + [i64] * 7 + [vp, i64, vp, vp, vp]
     L.oracle_mxfp4_decode.restype = ctypes.c_int
     L.oracle_mxfp4_decode.argtypes = [vp, vp, i64, i64, vp]
+    L.oracle_pool_keys_bf16.restype = ctypes.c_int
+    L.oracle_pool_keys_bf16.argtypes = [vp, i64, i64, i64, i64, vp]
+    L.oracle_topk_two_stage_bf16.restype = ctypes.c_int
+    L.oracle_topk_two_stage_bf16.argtypes = [vp, vp, vp] + [i64] * 9 + [vp, i64, vp, vp, vp]
     L.oracle_scores_bf16.restype = ctypes.c_int
     L.oracle_scores_bf16.argtypes = [vp, vp, vp] + [i64] * 6 + [i64, vp]
     if path is None:
@@ -109,6 +113,44 @@ def topk(q, kc, w, m: int, k: int, rows=None, q_scale=None, kc_scale=None, lib=N
         rc = L.oracle_topk_e4m3(q.ctypes.data, qs.ctypes.data, kc.ctypes.data, ks.ctypes.data,
                                 w.ctypes.data, B, S, T, H, D, m, k, rows.ctypes.data, n,
                                 idx.ctypes.data, sc.ctypes.data, sc64.ctypes.data)
+    if rc != 0:
+        raise ValueError(f"oracle returned {rc}")
+    return idx, sc, sc64
+
+
+def pool_keys(kc, G: int = 8, lib=None) -> np.ndarray:
+    """Pooled keys of the two-stage indexer: [B, T//G, D] float64 (bf16 values),
+    the mean of each block of G keys rounded once to bf16."""
+    L = lib or load()
+    kc = _c(kc, np.uint16)
+    B, T, D = kc.shape
+    out = np.empty((B, T // G, D), dtype=np.float64)
+    if T // G == 0:
+        return out
+    if L.oracle_pool_keys_bf16(kc.ctypes.data, B, T, D, G, out.ctypes.data) != 0:
+        raise ValueError("oracle_pool_keys_bf16 failed")
+    return out
+
+
+def topk_two_stage(q, kc, w, m: int, k: int, G: int = 8, n_keep: int = 2048, rows=None, lib=None):
+    """Two-stage oracle top-k (bf16 q [B,S,H,D], kc [B,T,D], w [B,S,H]): the
+    best n_keep complete visible blocks of G keys by the score of their pooled
+    key, then the top-k of their keys and the incomplete block's visible keys.
+    Returns (idx int32 [n,k], score float32 [n,k], score64 float64 [n,k])."""
+    L = lib or load()
+    B, S, H, D = q.shape
+    T = kc.shape[1]
+    if rows is None:
+        rows = np.arange(B * S, dtype=np.int64)
+    rows = _c(np.asarray(rows, dtype=np.int64), np.int64)
+    n = rows.shape[0]
+    idx = np.empty((n, k), dtype=np.int32)
+    sc = np.empty((n, k), dtype=np.float32)
+    sc64 = np.empty((n, k), dtype=np.float64)
+    q, kc, w = _c(q, np.uint16), _c(kc, np.uint16), _c(w, np.float32)
+    rc = L.oracle_topk_two_stage_bf16(q.ctypes.data, kc.ctypes.data, w.ctypes.data, B, S, T, H, D, m, k, G,
+                                      n_keep, rows.ctypes.data, n, idx.ctypes.data, sc.ctypes.data,
+                                      sc64.ctypes.data)
     if rc != 0:
         raise ValueError(f"oracle returned {rc}")
     return idx, sc, sc64

@@ -241,6 +241,121 @@ int oracle_topk_e4m3(const uint8_t* q, const float* q_scale, const uint8_t* kc,
   return topk_rows(&p, k, rows, n_rows, out_idx, out_score, out_score64);
 }
 
+/*
+ * Two-stage indexer (the V4.1-Flash indexer as the deployment notes describe
+ * it, "two-level sparse attention", indexer section: a cheap candidate stage
+ * first picks blocks of compressed keys -- 2048 blocks of 8 -- then the best
+ * keys among the candidates are kept).  The pages do not say how a block is
+ * scored; this oracle takes the plainest reading:
+ *   - block j of a sequence is keys jG .. jG+G-1 (nb = floor(T/G) blocks);
+ *   - its pooled key is the mean of its G keys rounded once to bf16 (nearest
+ *     even);
+ *   - the coarse score of block j for query t is the indexer score of the
+ *     pooled key; only complete visible blocks compete (jG+G-1 < n(t));
+ *   - the best n_keep blocks by (coarse score desc, block index asc) are
+ *     kept, all of them when fewer compete;
+ *   - the candidates are the keys of the kept blocks plus the visible keys
+ *     of the incomplete last block (n(t) mod G of them);
+ *   - the result is the top-k of the candidates by (indexer score desc, key
+ *     index asc), padded as the one-stage result.
+ * With at most n_keep complete visible blocks, every visible key is a
+ * candidate and the result is the one-stage top-k.
+ */
+
+/* Round to the nearest bf16 (ties to even), from double, for normal values. */
+static double round_bf16(double x) {
+  if (x == 0.0 || !isfinite(x)) return x;
+  int e;
+  frexp(x, &e);                 /* |x| = f * 2^e, f in [0.5, 1) */
+  double u = ldexp(1.0, e - 8); /* one unit in the 8th significant bit */
+  return nearbyint(x / u) * u;  /* default rounding mode: ties to even */
+}
+
+/* Pooled keys of sequence b: nb rows of D doubles (bf16 values). */
+static void pooled_keys(const problem_t* p, int64_t b, int64_t G, int64_t nb, double* pool, double* krow) {
+  for (int64_t j = 0; j < nb; ++j) {
+    for (int64_t d = 0; d < p->D; ++d) pool[j * p->D + d] = 0.0;
+    for (int64_t i = 0; i < G; ++i) {
+      widen_key(p, b, j * G + i, krow);
+      for (int64_t d = 0; d < p->D; ++d) pool[j * p->D + d] += krow[d];
+    }
+    for (int64_t d = 0; d < p->D; ++d) pool[j * p->D + d] = round_bf16(pool[j * p->D + d] / (double)G);
+  }
+}
+
+int oracle_pool_keys_bf16(const uint16_t* kc, int64_t B, int64_t T, int64_t D, int64_t G, double* out) {
+  if (B <= 0 || T <= 0 || D <= 0 || G <= 0) return -1;
+  problem_t p = {0, NULL, NULL, kc, NULL, NULL, B, 1, T, 1, D, 1, NULL};
+  double* krow = (double*)malloc(sizeof(double) * (size_t)D);
+  if (!krow) return -2;
+  int64_t nb = T / G;
+  for (int64_t b = 0; b < B; ++b) pooled_keys(&p, b, G, nb, out + b * nb * D, krow);
+  free(krow);
+  return 0;
+}
+
+int oracle_topk_two_stage_bf16(const uint16_t* q, const uint16_t* kc, const float* w, int64_t B, int64_t S,
+                               int64_t T, int64_t H, int64_t D, int64_t m, int64_t k, int64_t G,
+                               int64_t n_keep, const int64_t* rows, int64_t n_rows, int32_t* out_idx,
+                               float* out_score, double* out_score64) {
+  if (B <= 0 || S <= 0 || T <= 0 || H <= 0 || D <= 0 || m <= 0 || k <= 0 || G <= 0 || n_keep <= 0) return -1;
+  problem_t p = {0, q, NULL, kc, NULL, w, B, S, T, H, D, m, NULL};
+  const int64_t nb = T / G;
+  double* qrow = (double*)malloc(sizeof(double) * (size_t)(H * D));
+  double* wrow = (double*)malloc(sizeof(double) * (size_t)H);
+  double* krow = (double*)malloc(sizeof(double) * (size_t)D);
+  double* dot = (double*)malloc(sizeof(double) * (size_t)H);
+  double* pool = (double*)malloc(sizeof(double) * (size_t)((nb > 0 ? nb : 1) * D));
+  cand_t* blk = (cand_t*)malloc(sizeof(cand_t) * (size_t)(nb > 0 ? nb : 1));
+  cand_t* c = (cand_t*)malloc(sizeof(cand_t) * (size_t)T);
+  int rc = 0;
+  int64_t pooled_b = -1;
+  if (!qrow || !wrow || !krow || !dot || !pool || !blk || !c) rc = -2;
+  for (int64_t i = 0; rc == 0 && i < n_rows; ++i) {
+    int64_t r = rows[i];
+    if (r < 0 || r >= B * S) { rc = -1; break; }
+    int64_t b = r / S, t = r % S;
+    if (b != pooled_b) {
+      pooled_keys(&p, b, G, nb, pool, krow);
+      pooled_b = b;
+    }
+    int64_t n = oracle_visible_count(t, T, m);
+    int64_t nbv = n / G;
+    widen_query(&p, b, t, qrow, wrow);
+    /* coarse stage over the complete visible blocks */
+    for (int64_t j = 0; j < nbv; ++j) {
+      blk[j].score = score_rows(qrow, pool + j * D, wrow, (int)H, (int)D, dot);
+      blk[j].idx = j;
+    }
+    qsort(blk, (size_t)nbv, sizeof(cand_t), cand_cmp);
+    int64_t kept = nbv < n_keep ? nbv : n_keep;
+    /* fine stage over the kept blocks' keys and the incomplete block's visible keys */
+    int64_t nc = 0;
+    for (int64_t j = 0; j < kept; ++j)
+      for (int64_t e = 0; e < G; ++e) c[nc++].idx = blk[j].idx * G + e;
+    for (int64_t s = nbv * G; s < n; ++s) c[nc++].idx = s;
+    for (int64_t x = 0; x < nc; ++x) {
+      widen_key(&p, b, c[x].idx, krow);
+      c[x].score = score_rows(qrow, krow, wrow, (int)H, (int)D, dot);
+    }
+    qsort(c, (size_t)nc, sizeof(cand_t), cand_cmp);
+    for (int64_t j = 0; j < k; ++j) {
+      int64_t o = i * k + j;
+      if (j < nc) {
+        out_idx[o] = (int32_t)c[j].idx;
+        if (out_score) out_score[o] = (float)c[j].score;
+        if (out_score64) out_score64[o] = c[j].score;
+      } else {
+        out_idx[o] = -1;
+        if (out_score) out_score[o] = -INFINITY;
+        if (out_score64) out_score64[o] = -INFINITY;
+      }
+    }
+  }
+  free(qrow); free(wrow); free(krow); free(dot); free(pool); free(blk); free(c);
+  return rc;
+}
+
 /* All T scores of one row (bf16 inputs) in double; invisible keys get NaN.
  * For brute-force and invariant tests on small inputs. */
 int oracle_scores_bf16(const uint16_t* q, const uint16_t* kc, const float* w, int64_t B, int64_t S,

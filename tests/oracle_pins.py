@@ -245,5 +245,56 @@ def mxfp4_matches_bf16(lib):
     assert np.any(imx[:, 0] > 0)  # the keys are not all tied
 
 
+def two_stage_all_kept(lib):
+    """With at most n_keep complete visible blocks every visible key is a
+    candidate, so the two-stage result is the one-stage top-k (rows with an
+    incomplete last block included: S is not a multiple of m*G)."""
+    rng = np.random.default_rng(29)
+    B, S, T, H, D, m, k, G = 2, 300, 72, 3, 16, 4, 10, 8
+    q = _bits(rng.standard_normal((B, S, H, D)))
+    kc = _bits(rng.standard_normal((B, T, D)))
+    w = rng.random((B, S, H)).astype(np.float32)
+    i1, s1, _ = oracle.topk(q, kc, w, m, k, lib=lib)
+    for keep in (T // G, T // G + 5):
+        i2, s2, _ = oracle.topk_two_stage(q, kc, w, m, k, G=G, n_keep=keep, lib=lib)
+        assert np.array_equal(i1, i2) and np.array_equal(s1, s2), keep
+
+
+def two_stage_one_key_per_block(lib):
+    """Blocks with a single nonzero key (at a random position) and positive
+    values: a block's pooled key is that key / G exactly, its coarse score is
+    that key's score / G, so the kept blocks are those holding the n_keep best
+    keys and the two-stage top-n_keep equals the one-stage top-n_keep."""
+    rng = np.random.default_rng(31)
+    B, S, T, H, D, m, G, keep = 1, 400, 100, 2, 8, 4, 8, 5
+    q = _bits(rng.random((B, S, H, D)) + 0.25)
+    kc = np.zeros((B, T, D), dtype=np.float32)
+    pos = rng.integers(0, G, size=(B, (T + G - 1) // G))
+    for j in range(pos.shape[1]):
+        s = j * G + pos[0, j]
+        if s < T:
+            kc[0, s] = rng.random(D) + 0.25
+    kc = _bits(kc)
+    w = (rng.random((B, S, H)) + 0.1).astype(np.float32)
+    rows = np.arange(m * G * (keep + 1), S)  # rows with more than n_keep complete blocks
+    i1, s1, _ = oracle.topk(q, kc, w, m, keep, rows=rows, lib=lib)
+    i2, s2, _ = oracle.topk_two_stage(q, kc, w, m, keep, G=G, n_keep=keep, rows=rows, lib=lib)
+    assert np.all(s1 > 0)
+    assert np.array_equal(i1, i2) and np.array_equal(s1, s2)
+
+
+def two_stage_pooled_keys(lib):
+    """The pooled keys against numpy's block mean rounded to bf16 by
+    ml_dtypes (a library conversion, round to nearest even)."""
+    import ml_dtypes
+    rng = np.random.default_rng(37)
+    kc = _bits(rng.standard_normal((2, 70, 16)) * 3)
+    got = oracle.pool_keys(kc, 8, lib=lib)
+    blocks = _f(kc)[:, :64].reshape(2, 8, 8, 16)
+    want = blocks.mean(axis=2).astype(ml_dtypes.bfloat16).astype(np.float64)
+    assert got.shape == (2, 8, 16) and np.array_equal(got, want)
+
+
 ALL = [hand_cases, onehot_matmul, positive_closed, visible_closed, causal, prefix, brute_subsets,
-       invariances, batch_independent, fp8_matches_bf16, mxfp4_matches_bf16]
+       invariances, batch_independent, fp8_matches_bf16, mxfp4_matches_bf16, two_stage_all_kept,
+       two_stage_one_key_per_block, two_stage_pooled_keys]

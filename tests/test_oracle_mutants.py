@@ -37,6 +37,14 @@ MUTANTS = {
                            "(d & 1) ? (uint8_t)(byte & 15) : (uint8_t)(byte >> 4)"),
     "mx_one_scale_per_row": ("scales[r * (D / 32) + d / 32]", "scales[r * (D / 32)]"),
     "e8m0_bias126": ("return ldexp(1.0, (int)bits - 127);", "return ldexp(1.0, (int)bits - 126);"),
+    "pool_first_keys_only": ("for (int64_t i = 0; i < G; ++i) {\n      widen_key(p, b, j * G + i, krow);",
+                             "for (int64_t i = 0; i < G - 1; ++i) {\n      widen_key(p, b, j * G + i, krow);"),
+    "pool_no_bf16_rounding": ("= round_bf16(pool[j * p->D + d] / (double)G);", "= pool[j * p->D + d] / (double)G;"),
+    "two_stage_no_tail": ("for (int64_t s = nbv * G; s < n; ++s) c[nc++].idx = s;", ""),
+    "two_stage_keep_one_less": ("int64_t kept = nbv < n_keep ? nbv : n_keep;",
+                                "int64_t kept = nbv < n_keep - 1 ? nbv : n_keep - 1;"),
+    "two_stage_worst_blocks": ("c[nc++].idx = blk[j].idx * G + e;", "c[nc++].idx = blk[nbv - 1 - j].idx * G + e;"),
+    "two_stage_incomplete_block": ("int64_t nbv = n / G;", "int64_t nbv = (n + G - 1) / G < nb ? (n + G - 1) / G : nb;"),
 }
 
 RUNNER = r"""
