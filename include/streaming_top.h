@@ -170,6 +170,38 @@ SI_API si_status si_indexer_materialize_noalloc(const void* q, const void* kc, c
                                                 int32_t* out_idx, float* out_score, void* stream);
 
 /*
+ * Two-stage indexer top-k: the V4.1-Flash indexer as its deployment notes
+ * describe it ("two-level sparse attention", indexer section): a cheap
+ * candidate stage picks, per query, n_keep blocks of `block` compressed keys
+ * (the notes: 2048 blocks of 8), then the top-k of the candidates is kept
+ * (the notes: 512).  Reading of what the pages leave open:
+ *   - block j is keys j*block .. j*block+block-1 (floor(T/block) blocks);
+ *     its pooled key is the mean of its keys rounded once to bf16;
+ *   - a block competes for query t once all its keys are visible; the
+ *     n_keep best by the indexer score of the pooled key are kept (all of
+ *     them when fewer compete; ties to the lower block);
+ *   - the candidates are the kept blocks' keys and the visible keys of the
+ *     incomplete last block; the result is their top-k by the indexer score,
+ *     exactly as si_indexer_topk orders and pads it.
+ * With at most n_keep complete visible blocks the result is si_indexer_topk's.
+ *   q [B,S,H_I,D] bf16, kc [B,T,D] bf16, w [B,S,H_I] fp32 (device);
+ *   out_idx, out_score [B,S,k] (device, written; out_score required).
+ * Supported: bf16 (opt->dtype 0 or opt NULL), D == 128, H_I == 64,
+ * 1 <= k <= 2048, 1 <= n_keep <= 2048, 1 <= block <= 64; else
+ * SI_ERR_UNSUPPORTED / SI_ERR_INVALID_ARGUMENT.  Rows are processed in
+ * chunks of opt->query_chunk rows (0 = 16384); scratch of
+ * si_two_stage_workspace_size() bytes comes from opt->workspace when given,
+ * else it is allocated and freed on `stream`.  Asynchronous on `stream`.
+ */
+SI_API si_status si_indexer_topk_two_stage(const void* q, const void* kc, const float* w, int B, int S, int T,
+                                           int H_I, int D, int m, int k, int block, int n_keep,
+                                           int32_t* out_idx, float* out_score, void* stream,
+                                           const si_options* opt);
+
+/* Scratch bytes of si_indexer_topk_two_stage (query_chunk 0 = 16384). */
+SI_API size_t si_two_stage_workspace_size(int B, int S, int T, int block, int n_keep, int query_chunk);
+
+/*
  * Decodes MXFP4 rows to bf16: codes [rows, D/2] bytes (value d in the low
  * nibble of byte d/2 when d is even, the high nibble when odd), E8M0 scales
  * [rows, D/32] (one per 32 values), out [rows, D] bf16; device pointers,

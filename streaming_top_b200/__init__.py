@@ -56,6 +56,10 @@ _lib.si_indexer_materialize_noalloc.argtypes = _ARGS
 NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024  # SI_NOALLOC_SCRATCH_BYTES
 _lib.si_indexer_workspace_size.restype = _sz
 _lib.si_indexer_workspace_size.argtypes = [_i] * 8 + [ctypes.POINTER(Options)]
+_lib.si_indexer_topk_two_stage.restype = _i
+_lib.si_indexer_topk_two_stage.argtypes = [_vp, _vp, _vp] + [_i] * 9 + [_vp, _vp, _vp, ctypes.POINTER(Options)]
+_lib.si_two_stage_workspace_size.restype = _sz
+_lib.si_two_stage_workspace_size.argtypes = [_i] * 6
 _lib.si_mxfp4_to_bf16.restype = _i
 _lib.si_mxfp4_to_bf16.argtypes = [_vp, _vp, ctypes.c_int64, _i, _vp, _vp]
 _lib.si_device_status.restype = _i
@@ -190,6 +194,26 @@ def indexer_topk_rows(q, kc, w, m: int, k: int, row0: int, *, q_scale=None, kc_s
                                    _stream_ptr(stream), ctypes.byref(o))
     _check(st, "si_indexer_topk_rows")
     return out_idx, out_score
+
+
+def indexer_topk_two_stage(q, kc, w, m: int, k: int, *, block: int = 8, n_keep: int = 2048,
+                           query_chunk: int = 0, out_idx=None, out_score=None, workspace=None, stream=None):
+    """Two-stage indexer top-k (``si_indexer_topk_two_stage``): the best
+    n_keep blocks of `block` keys by the score of their pooled (mean) key,
+    then the top-k of their keys and the incomplete block's visible keys.
+    Returns (idx, score) [B, S, k], ordered as indexer_topk's."""
+    B, S, T, H, D = _shapes(q, kc, w)
+    out_idx, out_score = _outputs(B, S, k, q.device, out_idx, out_score, True)
+    o = _options(q, kc, None, None, query_chunk, 0, workspace)
+    st = _lib.si_indexer_topk_two_stage(q.data_ptr(), kc.data_ptr(), w.data_ptr(), B, S, T, H, D, m, k,
+                                        int(block), int(n_keep), out_idx.data_ptr(), out_score.data_ptr(),
+                                        _stream_ptr(stream), ctypes.byref(o))
+    _check(st, "si_indexer_topk_two_stage")
+    return out_idx, out_score
+
+
+def two_stage_workspace_size(B, S, T, block=8, n_keep=2048, query_chunk=0) -> int:
+    return int(_lib.si_two_stage_workspace_size(B, S, T, block, n_keep, query_chunk))
 
 
 def mxfp4_to_bf16(codes, scales, out=None, stream=None):

@@ -267,6 +267,31 @@ size_t si_indexer_workspace_size(int B, int S, int T, int H_I, int D, int m, int
   return opt && opt->dtype == SI_DTYPE_MXFP4_KEYS ? mxfp4_key_bytes(B, T, D) : 0;
 }
 
+size_t si_two_stage_workspace_size(int B, int S, int T, int block, int n_keep, int query_chunk) {
+  if (B < 1 || S < 1 || T < 1 || block < 1 || n_keep < 1 || query_chunk < 0) return 0;
+  return two_stage_workspace_bytes(B, S, T, block, n_keep, query_chunk ? query_chunk : 16384);
+}
+
+si_status si_indexer_topk_two_stage(const void* q, const void* kc, const float* w, int B, int S, int T,
+                                    int H_I, int D, int m, int k, int block, int n_keep, int32_t* out_idx,
+                                    float* out_score, void* stream, const si_options* opt) {
+  si_status st = check_common(q, kc, w, B, S, T, H_I, D, m, k, out_idx, out_score);
+  if (st != SI_OK) return st;
+  if (!out_score) return fail(SI_ERR_INVALID_ARGUMENT, "the two-stage path needs out_score");
+  if (opt && opt->dtype != SI_DTYPE_BF16) return fail(SI_ERR_UNSUPPORTED, "the two-stage path takes bf16 inputs");
+  if (block < 1 || block > 64 || n_keep < 1 || n_keep > 2048)
+    return fail(SI_ERR_INVALID_ARGUMENT, "1 <= block <= 64 and 1 <= n_keep <= 2048 (got %d, %d)", block, n_keep);
+  if (D != 128 || H_I != 64)
+    return fail(SI_ERR_UNSUPPORTED, "two-stage path implements D=128, H_I=64 (got D=%d, H_I=%d)", D, H_I);
+  if (k > 2048) return fail(SI_ERR_UNSUPPORTED, "k <= 2048 (got %d)", k);
+  if (static_cast<long long>(m) * block > 0x7FFFFFFFll || static_cast<long long>(B) * S * H_I > 0x7FFFFFFFll)
+    return fail(SI_ERR_UNSUPPORTED, "m*block and B*S*H_I must fit in 31 bits");
+  const int chunk = opt && opt->query_chunk > 0 ? opt->query_chunk : 16384;
+  return launch_two_stage(q, kc, w, B, S, T, m, k, block, n_keep, chunk, out_idx, out_score,
+                          opt ? opt->workspace : nullptr, opt ? opt->workspace_bytes : 0, kDefaultWaitLimitNs,
+                          static_cast<cudaStream_t>(stream));
+}
+
 si_status si_mxfp4_to_bf16(const void* codes, const void* scales, int64_t rows, int D, void* out,
                            void* stream) {
   if (rows < 0) return fail(SI_ERR_INVALID_ARGUMENT, "rows must be >= 0 (got %lld)", static_cast<long long>(rows));

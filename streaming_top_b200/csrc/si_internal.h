@@ -46,6 +46,13 @@ struct StreamConfig {
 si_status launch_mxfp4_to_bf16(const void* codes, const void* scales, long long rows, int D, void* out,
                                cudaStream_t stream);
 
+// Two-stage indexer (blocks of G keys scored by their pooled key, the best
+// n_keep kept, then the top-k of their keys): scratch bytes and driver.
+size_t two_stage_workspace_bytes(int B, int S, int T, int G, int n_keep, int chunk);
+si_status launch_two_stage(const void* q, const void* kc, const float* w, int B, int S, int T, int m, int k,
+                           int G, int n_keep, int chunk, int32_t* out_idx, float* out_score, void* workspace,
+                           size_t workspace_bytes, uint64_t wait_limit_ns, cudaStream_t stream);
+
 // Sorts rows [rows, k] of (idx, score) in place by (score desc, index asc).
 si_status launch_row_sort(int32_t* idx, float* score, long long rows, int k, cudaStream_t stream);
 

@@ -157,3 +157,18 @@ class _Cuda:
 
     def data_ptr(self):
         return self._t.data_ptr()
+
+
+def test_two_stage_validation():
+    L = si.lib()
+    args = [P, P, P, 1, 64, 64, 64, 128, 4, 8]
+    assert L.si_indexer_topk_two_stage(*args, 0, 16, P, P, None, None) == si.SI_ERR_INVALID_ARGUMENT  # block 0
+    assert L.si_indexer_topk_two_stage(*args, 8, 4096, P, P, None, None) == si.SI_ERR_INVALID_ARGUMENT
+    assert L.si_indexer_topk_two_stage(*args, 8, 16, P, None, None, None) == si.SI_ERR_INVALID_ARGUMENT
+    o = si.Options()
+    o.dtype = si.SI_DTYPE_FP8_E4M3
+    assert L.si_indexer_topk_two_stage(*args, 8, 16, P, P, None, ctypes.byref(o)) == si.SI_ERR_UNSUPPORTED
+    assert L.si_indexer_topk_two_stage(P, P, P, 1, 64, 64, 32, 128, 4, 8, 8, 16, P, P, None, None) == \
+        si.SI_ERR_UNSUPPORTED  # H_I = 32
+    assert si.two_stage_workspace_size(1, 64, 64, 8, 16, 0) > 0
+    assert si.two_stage_workspace_size(1, 64, 64, 0, 16, 0) == 0
