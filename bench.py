@@ -156,9 +156,29 @@ def job_value(world: int, pairs_per_rank: int, ms_step: float) -> float:
     return world * pairs_per_rank / (ms_step * 1e-3)
 
 
-def oracle_sample(wl, inp, rows) -> tuple[float, int]:
+TWO_STAGE = {"block": 8, "n_keep": 2048}  # the V4.1-Flash indexer's candidate stage: 2048 blocks of 8
+TWO_STAGE_CHUNK = 65536
+
+
+def two_stage_pairs(wl) -> tuple[int, int]:
+    """(coarse pairs, fine pairs) the two-stage path scores: per row, the
+    complete visible blocks, and the kept blocks' keys plus the incomplete
+    block's visible keys."""
+    t = np.arange(wl.S, dtype=np.int64)
+    n = np.minimum(wl.T, (t + 1) // wl.m)
+    nbv = n // TWO_STAGE["block"]
+    fine = np.minimum(nbv, TWO_STAGE["n_keep"]) * TWO_STAGE["block"] + (n - nbv * TWO_STAGE["block"])
+    return wl.B * int(nbv.sum()), wl.B * int(fine.sum())
+
+
+def oracle_sample(wl, inp, rows, two_stage: bool = False) -> tuple[float, int]:
     import oracle
     t0 = time.perf_counter()
+    if two_stage:
+        oracle.topk_two_stage(inp["q"], inp["kc"], inp["w"], wl.m, wl.k, G=TWO_STAGE["block"],
+                              n_keep=TWO_STAGE["n_keep"], rows=rows)
+        dt = time.perf_counter() - t0
+        return dt, int(sum(min(wl.T, (int(r) % wl.S + 1) // wl.m) for r in rows))
     oracle.topk(inp["q"], inp["kc"], inp["w"], wl.m, wl.k, rows=rows, q_scale=inp.get("q_scale"),
                 kc_scale=inp.get("kc_scale"), kc_mx_scale=inp.get("kc_mx_scale"))
     dt = time.perf_counter() - t0
@@ -178,7 +198,7 @@ def run_reference(args, wl):
     times, pairs = [], []
     for i in range(args.warmup + args.steps):
         rows = np.sort(allrows[i * per_step:(i + 1) * per_step])
-        dt, pr = oracle_sample(wl, inp, rows)
+        dt, pr = oracle_sample(wl, inp, rows, args.method == "two-stage")
         if i >= args.warmup:
             times.append(dt)
             pairs.append(pr)
@@ -224,6 +244,9 @@ def run_ours(args, wl):
     fp8 = args.fmt == "e4m3"
     mx = args.fmt == "mxfp4"  # bf16 queries, MXFP4 keys (decoded to bf16 inside the call)
     rows_mode = args.shard == "rows"
+    two = args.method == "two-stage"
+    if two and (args.fmt != "bf16" or rows_mode):
+        raise SystemExit("--method two-stage runs bf16 inputs over whole sequences")
     if rows_mode:
         # every rank holds the same sequences' keys and weights and only its
         # own query rows (equal visible pairs per rank)
@@ -263,6 +286,13 @@ def run_ours(args, wl):
     # streaming kernel (rows left unsorted), then the row sort; an event
     # between them times the streaming kernel alone for the roofline
     def step(mid=None):
+        if two:
+            # one si_indexer_topk_two_stage call (pool, coarse, fine, select, row sort)
+            si.indexer_topk_two_stage(q, kc, w, wl.m, wl.k, query_chunk=TWO_STAGE_CHUNK, out_idx=out_idx,
+                                      out_score=out_score, stream=stream, **TWO_STAGE)
+            if mid is not None:
+                mid.record(stream)
+            return
         if rows_mode:
             si.indexer_topk_rows(q, kc, w, wl.m, wl.k, r0, q_scale=qs, kc_scale=ks, out_idx=out_idx,
                                  out_score=out_score, unsorted=True, stream=stream, kc_mx_scale=kms)
@@ -319,7 +349,8 @@ def run_ours(args, wl):
     bufs = {}
     for _ in range(max(1, args.warmup)):
         si.indexer_topk_host(hq, hk, hw, wl.m, wl.k, q_scale=hqs, kc_scale=hks, device=dev, bufs=bufs,
-                             row0=r0, kc_mx_scale=hkms)
+                             row0=r0, kc_mx_scale=hkms, two_stage=TWO_STAGE if two else None,
+                             query_chunk=TWO_STAGE_CHUNK if two else 0)
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
     if world > 1:
@@ -328,7 +359,8 @@ def run_ours(args, wl):
     for e0, e1 in e2e_ev:
         e0.record(stream)
         si.indexer_topk_host(hq, hk, hw, wl.m, wl.k, q_scale=hqs, kc_scale=hks, device=dev, bufs=bufs,
-                             sync=False, row0=r0, kc_mx_scale=hkms)
+                             sync=False, row0=r0, kc_mx_scale=hkms, two_stage=TWO_STAGE if two else None,
+                             query_chunk=TWO_STAGE_CHUNK if two else 0)
         e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev) / args.steps
@@ -361,9 +393,13 @@ def run_ours(args, wl):
         e2e_value = job_value(world, P, e2e_ms)
     tflops = P * flop_pair / (ms_step * 1e-3) / 1e12
     kernel_tflops = P * flop_pair / (ms_kernel * 1e-3) / 1e12
+    if two:
+        # the pairs the two stages actually score (pooled keys, then candidates)
+        cp, fpairs = two_stage_pairs(wl)
+        kernel_tflops = (cp + fpairs) * flop_pair / (ms_kernel * 1e-3) / 1e12
     alg_bytes = nbytes(q, kc, w, out_idx, out_score, qs, ks, kms)
     # the committed DRAM capture is of the whole-sequence bf16 launch
-    traffic = None if fp8 or mx or (rows_mode and world > 1) else ncu_traffic(wl.name)
+    traffic = None if fp8 or mx or two or (rows_mode and world > 1) else ncu_traffic(wl.name)
     # a contraction is measured against the peak of its own type: fp8 takes the
     # measured bf16 matmul peak times the nominal fp8 / bf16 ratio (4.5 / 2.25)
     peak_tc = peaks["bf16_tflops"] * (2.0 if fp8 else 1.0)
@@ -377,7 +413,7 @@ def run_ours(args, wl):
         done, t_tot, p_tot = 0, 0.0, 0
         while t_tot < args.cpu_seconds and done < len(rows):
             chunk = np.sort(rows[done:done + 16])
-            dt, pr = oracle_sample(wl, inp, chunk)
+            dt, pr = oracle_sample(wl, inp, chunk, two)
             t_tot += dt
             p_tot += pr
             done += len(chunk)
@@ -391,7 +427,12 @@ def run_ours(args, wl):
         "vs_baseline": None, "dtype": "bf16" if mx else args.fmt, "data": "synthetic",
         "config": dict(config_dict(wl, world, args.shard, bounds),
                        **({"keys": "MXFP4 (E2M1 codes, E8M0 scale per 32 values), decoded to bf16 "
-                                   "inside the call"} if mx else {})),
+                                   "inside the call"} if mx else {}),
+                       **({"method": f"two-stage: the best {TWO_STAGE['n_keep']} blocks of {TWO_STAGE['block']} "
+                                     f"keys by their pooled key, then the top-{wl.k} of their keys; value counts "
+                                     "the workload's visible pairs, the roofline the pairs the two stages score "
+                                     f"({two_stage_pairs(wl)[0]} pooled + {two_stage_pairs(wl)[1]} candidate)",
+                           "query_chunk": TWO_STAGE_CHUNK} if two else {})),
         "tflops": tflops,
         "frac_bf16_peak": tflops / peaks["bf16_tflops"],
         "frac_bf16_peak_sustained": tflops / peaks["bf16_tflops_sustained"] if peaks["bf16_tflops_sustained"] else None,
@@ -402,8 +443,12 @@ def run_ours(args, wl):
                              "out_idx": nbytes(out_idx) / 1e9, "out_score": nbytes(out_score) / 1e9,
                              "l2_flush_buffer": flush.numel() / 1e9,
                              "library_workspace": (wl.B * wl.T * wl.D * 2 + 256) / 1e9 if mx else 0.0},
-        "kernel_ms": {"stream_topk_kernel": ms_kernel, "row_sort_kernel": ms_sort},
-        "roofline": {"bound": "tensor", "kernel": "stream_topk_kernel", "achieved": kernel_tflops,
+        "kernel_ms": ({"indexer_topk_two_stage call": ms_kernel} if two else
+                      {"stream_topk_kernel": ms_kernel, "row_sort_kernel": ms_sort}),
+        "roofline": {"bound": "tensor",
+                     "kernel": ("two-stage call (pool, coarse stream_topk_kernel, fine_score_kernel, select, "
+                                "row sort)" if two else "stream_topk_kernel"),
+                     "achieved": kernel_tflops,
                      "peak": peak_tc, "unit": "TFLOP/s",
                      "frac": kernel_tflops / peak_tc,
                      "peak_source": peak_src,
@@ -411,7 +456,7 @@ def run_ours(args, wl):
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "pairs/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": ((2 + 3 * wl.B * -(-wl.S // TWO_STAGE_CHUNK)) if two else 2) * args.steps,
         "clocks": clocks,
         "wall_s_timed": wall,
     }
@@ -431,6 +476,9 @@ def main() -> int:
                     help="input format: bf16 (default), fp8 e4m3 with per-row scales, or mxfp4 keys "
                          "(E2M1 + E8M0 per 32 values) with bf16 queries")
     ap.add_argument("--ref-rows", type=int, default=32)
+    ap.add_argument("--method", default="one-stage", choices=["one-stage", "two-stage"],
+                    help="one-stage (the streaming top-k over all visible keys) or the two-stage indexer "
+                         "(2048 blocks of 8 kept by their pooled key, then the top-k of their keys)")
     ap.add_argument("--shard", default="seq", choices=["seq", "rows"],
                     help="N>1: independent sequences per GPU (seq, weak scaling) or the same sequences' "
                          "query rows split over the GPUs at equal visible pairs (rows, strong scaling)")

@@ -291,13 +291,15 @@ def device_status(stream=None) -> int:
 
 def indexer_topk_host(q, kc, w, m: int, k: int, *, q_scale=None, kc_scale=None, device="cuda",
                       query_chunk: int = 0, key_tile: int = 0, bufs: dict | None = None,
-                      sync: bool = True, row0: int | None = None, kc_mx_scale=None):
+                      sync: bool = True, row0: int | None = None, kc_mx_scale=None,
+                      two_stage: dict | None = None):
     """End-to-end call on HOST tensors (pinned for best speed): copies the
     inputs to the device, runs the streaming top-k, copies (idx, score) back.
     `bufs` may hold reusable device buffers from a previous call.  With
     sync=False the copies back are only enqueued on the current stream.
     With `row0`, q and w hold only rows row0 .. row0+R-1 of the sequences
-    (si_indexer_topk_rows)."""
+    (si_indexer_topk_rows).  With `two_stage` (keyword arguments of
+    indexer_topk_two_stage: block, n_keep), the two-stage indexer runs."""
     bufs = {} if bufs is None else bufs
     stream = torch.cuda.current_stream(device)
 
@@ -319,7 +321,10 @@ def indexer_topk_host(q, kc, w, m: int, k: int, *, q_scale=None, kc_scale=None, 
     if oi is None or oi.shape != (B, S, k):
         oi = bufs["out_idx"] = torch.empty((B, S, k), dtype=torch.int32, device=device)
         os_ = bufs["out_score"] = torch.empty((B, S, k), dtype=torch.float32, device=device)
-    if row0 is None:
+    if two_stage is not None:
+        indexer_topk_two_stage(qd, kd, wd, m, k, query_chunk=query_chunk, out_idx=oi, out_score=os_,
+                               stream=stream, **two_stage)
+    elif row0 is None:
         indexer_topk(qd, kd, wd, m, k, q_scale=qs, kc_scale=ks, query_chunk=query_chunk,
                      key_tile=key_tile, out_idx=oi, out_score=os_, stream=stream, kc_mx_scale=kms)
     else:
