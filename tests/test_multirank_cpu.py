@@ -146,3 +146,30 @@ def test_row_shards_balance_and_cover():
             p = [si.visible_pairs_before(y, T, m) - si.visible_pairs_before(x, T, m) for x, y in zip(b, b[1:])]
             if S >= 65536:
                 assert max(p) / min(p) < 1.001
+
+
+def test_two_stage_pair_counts_match_brute_force():
+    """bench's count of the pairs the two stages score (complete visible
+    blocks, then kept blocks' keys plus the incomplete block's visible keys)
+    against a row-by-row count, on a shape where the block budget binds."""
+    import dataclasses
+    wl = dataclasses.replace(synth.WORKLOADS["tiny"], S=70000)
+    cp, fp = bench.two_stage_pairs(wl)
+    G, keep = bench.TWO_STAGE["block"], bench.TWO_STAGE["n_keep"]
+    c_bf = f_bf = 0
+    for t in range(wl.S):
+        n = min(wl.T, (t + 1) // wl.m)
+        c_bf += n // G
+        f_bf += min(n // G, keep) * G + n % G
+    assert (cp, fp) == (c_bf, f_bf)
+    assert fp < synth.visible_pairs(wl.S, wl.T, wl.m)
+
+
+def test_reference_arm_two_stage_line():
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                        "--warmup", "0", "--workload", "tiny", "--method", "two-stage", "--ref-rows", "8"],
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    import json
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["value"] > 0 and line["cpu_baseline"]["kind"] == "oracle"
