@@ -61,6 +61,8 @@ def load(path: str | None = None):
     L.oracle_pool_keys_bf16.argtypes = [vp, i64, i64, i64, i64, vp]
     L.oracle_topk_two_stage_bf16.restype = ctypes.c_int
     L.oracle_topk_two_stage_bf16.argtypes = [vp, vp, vp] + [i64] * 9 + [vp, i64, vp, vp, vp]
+    L.oracle_sparse_attention_bf16.restype = ctypes.c_int
+    L.oracle_sparse_attention_bf16.argtypes = [vp, vp, vp] + [i64] * 7 + [ctypes.c_double, vp, vp]
     L.oracle_scores_bf16.restype = ctypes.c_int
     L.oracle_scores_bf16.argtypes = [vp, vp, vp] + [i64] * 6 + [i64, vp]
     if path is None:
@@ -154,6 +156,26 @@ def topk_two_stage(q, kc, w, m: int, k: int, G: int = 8, n_keep: int = 2048, row
     if rc != 0:
         raise ValueError(f"oracle returned {rc}")
     return idx, sc, sc64
+
+
+def sparse_attention(q, kv, idx, dv: int, scale: float | None = None, lib=None):
+    """Sparse attention over selected compressed entries: q [B,S,H,Dk] and
+    kv [B,T,Dk] bf16 bits, idx [B,S,k] int32 (-1 = padding); every head
+    attends over kv[idx] as keys (all Dk) and values (the first dv).
+    scale defaults to 1/sqrt(Dk).  Returns (out float64 [B,S,H,dv], lse
+    float64 [B,S,H])."""
+    L = lib or load()
+    q, kv, idx = _c(q, np.uint16), _c(kv, np.uint16), _c(idx, np.int32)
+    B, S, H, Dk = q.shape
+    T, k = kv.shape[1], idx.shape[2]
+    scale = 1.0 / np.sqrt(Dk) if scale is None else float(scale)
+    out = np.empty((B, S, H, dv), dtype=np.float64)
+    lse = np.empty((B, S, H), dtype=np.float64)
+    rc = L.oracle_sparse_attention_bf16(q.ctypes.data, kv.ctypes.data, idx.ctypes.data, B, S, T, H, Dk, dv, k,
+                                        scale, out.ctypes.data, lse.ctypes.data)
+    if rc != 0:
+        raise ValueError(f"oracle returned {rc}")
+    return out, lse
 
 
 def mxfp4_decode(codes, scales, lib=None) -> np.ndarray:

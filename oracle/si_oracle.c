@@ -356,6 +356,67 @@ int oracle_topk_two_stage_bf16(const uint16_t* q, const uint16_t* kc, const floa
   return rc;
 }
 
+/*
+ * Sparse attention over the selected compressed entries: the consumer of the
+ * indexer's top-k in the CSA pipeline (StreamIndex abstract: a sparse
+ * attention kernel reads only the selected entries).  The pages give no
+ * dimensions for it; the reading follows the DeepSeek-V3.2 lineage they
+ * name: every head of query t attends over the compressed latents idx[t, j]
+ * (index -1 = padding, skipped), each latent serving as key (all Dk values)
+ * and as value (its first Dv values):
+ *   o[t,h,:] = sum_j p_j kv[idx_j, :Dv],  p = softmax_j(scale * q[t,h,:] . kv[idx_j, :])
+ * and lse[t,h] = log sum_j exp(scale * logit_j) (-inf and o = 0 when no
+ * entry is valid).  fp64 throughout; the maximum logit is subtracted before
+ * exponentiating.
+ *   q [B,S,H,Dk] bf16, kv [B,T,Dk] bf16, idx [B,S,k] int32; out [B,S,H,Dv]
+ *   and lse [B,S,H] double.  Returns 0, -1 on a bad argument or index.
+ */
+int oracle_sparse_attention_bf16(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int64_t B,
+                                 int64_t S, int64_t T, int64_t H, int64_t Dk, int64_t Dv, int64_t k,
+                                 double scale, double* out, double* lse) {
+  if (B <= 0 || S <= 0 || T <= 0 || H <= 0 || Dk <= 0 || Dv <= 0 || Dv > Dk || k <= 0) return -1;
+  double* logit = (double*)malloc(sizeof(double) * (size_t)k);
+  if (!logit) return -2;
+  int rc = 0;
+  for (int64_t b = 0; b < B && rc == 0; ++b)
+    for (int64_t t = 0; t < S && rc == 0; ++t) {
+      const int32_t* sel = idx + (b * S + t) * k;
+      for (int64_t j = 0; j < k; ++j)
+        if (sel[j] < -1 || sel[j] >= T) rc = -1;
+      if (rc) break;
+      for (int64_t h = 0; h < H; ++h) {
+        const uint16_t* qh = q + ((b * S + t) * H + h) * Dk;
+        double* o = out + ((b * S + t) * H + h) * Dv;
+        double mx = -INFINITY;
+        for (int64_t j = 0; j < k; ++j) {
+          if (sel[j] < 0) continue;
+          const uint16_t* kr = kv + (b * T + sel[j]) * Dk;
+          double dot = 0.0;
+          for (int64_t d = 0; d < Dk; ++d) dot += oracle_bf16_value(qh[d]) * oracle_bf16_value(kr[d]);
+          logit[j] = scale * dot;
+          if (logit[j] > mx) mx = logit[j];
+        }
+        for (int64_t d = 0; d < Dv; ++d) o[d] = 0.0;
+        if (mx == -INFINITY) {
+          lse[(b * S + t) * H + h] = -INFINITY;
+          continue;
+        }
+        double den = 0.0;
+        for (int64_t j = 0; j < k; ++j) {
+          if (sel[j] < 0) continue;
+          const double e = exp(logit[j] - mx);
+          den += e;
+          const uint16_t* vr = kv + (b * T + sel[j]) * Dk;
+          for (int64_t d = 0; d < Dv; ++d) o[d] += e * oracle_bf16_value(vr[d]);
+        }
+        for (int64_t d = 0; d < Dv; ++d) o[d] /= den;
+        lse[(b * S + t) * H + h] = mx + log(den);
+      }
+    }
+  free(logit);
+  return rc;
+}
+
 /* All T scores of one row (bf16 inputs) in double; invisible keys get NaN.
  * For brute-force and invariant tests on small inputs. */
 int oracle_scores_bf16(const uint16_t* q, const uint16_t* kc, const float* w, int64_t B, int64_t S,

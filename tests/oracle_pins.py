@@ -295,6 +295,67 @@ def two_stage_pooled_keys(lib):
     assert got.shape == (2, 8, 16) and np.array_equal(got, want)
 
 
+def _attn_problem(rng, B=2, S=5, T=12, H=3, Dk=16, k=6):
+    q = _bits(rng.standard_normal((B, S, H, Dk)))
+    kv = _bits(rng.standard_normal((B, T, Dk)))
+    idx = np.stack([np.stack([rng.permutation(T)[:k] for _ in range(S)]) for _ in range(B)]).astype(np.int32)
+    idx[0, 1, 4:] = -1   # padding
+    idx[1, 2, :] = -1    # a row with nothing selected
+    return q, kv, idx
+
+
+def attn_matches_sdpa(lib):
+    """Sparse attention against torch's scaled_dot_product_attention (fp64,
+    CPU) over each query's gathered entries, and lse against logsumexp."""
+    import torch
+    rng = np.random.default_rng(41)
+    q, kv, idx = _attn_problem(rng)
+    Dv = 10
+    out, lse = oracle.sparse_attention(q, kv, idx, Dv, lib=lib)
+    Q, KV = torch.from_numpy(_f(q)), torch.from_numpy(_f(kv))
+    B, S, H, Dk = q.shape
+    for b in range(B):
+        for t in range(S):
+            sel = [int(x) for x in idx[b, t] if x >= 0]
+            if not sel:
+                assert np.all(out[b, t] == 0) and np.all(np.isneginf(lse[b, t]))
+                continue
+            K = KV[b, sel]                       # [n, Dk]
+            want = torch.nn.functional.scaled_dot_product_attention(
+                Q[b, t][:, None, :], K[None].expand(H, -1, -1), K[None, :, :Dv].expand(H, -1, -1))[:, 0]
+            assert np.allclose(out[b, t], want.numpy(), rtol=1e-12, atol=1e-13)
+            want_lse = torch.logsumexp((Q[b, t] @ K.T) / np.sqrt(Dk), dim=-1)
+            assert np.allclose(lse[b, t], want_lse.numpy(), rtol=1e-12, atol=1e-13)
+
+
+def attn_special_cases(lib):
+    """One selected entry gives exactly its value rows (weight 1); all-zero
+    queries give the plain mean of the selected values; permuting the
+    selection and moving the padding changes nothing beyond rounding."""
+    rng = np.random.default_rng(43)
+    q, kv, idx = _attn_problem(rng)
+    Dv = 16
+    one = np.full_like(idx, -1)
+    one[:, :, 2] = idx[:, :, 0].clip(0)
+    out, lse = oracle.sparse_attention(q, kv, one, Dv, lib=lib)
+    vals = _f(kv)
+    for b in range(q.shape[0]):
+        for t in range(q.shape[1]):
+            assert np.array_equal(out[b, t], np.broadcast_to(vals[b, one[b, t, 2], :Dv], out[b, t].shape))
+    zq = np.zeros_like(q)
+    out0, _ = oracle.sparse_attention(zq, kv, idx, Dv, lib=lib)
+    for b in range(q.shape[0]):
+        for t in range(q.shape[1]):
+            sel = [int(x) for x in idx[b, t] if x >= 0]
+            if sel:
+                assert np.allclose(out0[b, t], vals[b, sel, :Dv].mean(axis=0), rtol=1e-14, atol=1e-15)
+    perm = idx[:, :, ::-1].copy()
+    out_p, lse_p = oracle.sparse_attention(q, kv, perm, Dv, lib=lib)
+    out_r, lse_r = oracle.sparse_attention(q, kv, idx, Dv, lib=lib)
+    assert np.allclose(out_p, out_r, rtol=1e-12, atol=1e-14)
+    assert np.allclose(lse_p[np.isfinite(lse_r)], lse_r[np.isfinite(lse_r)], rtol=1e-13)
+
+
 ALL = [hand_cases, onehot_matmul, positive_closed, visible_closed, causal, prefix, brute_subsets,
        invariances, batch_independent, fp8_matches_bf16, mxfp4_matches_bf16, two_stage_all_kept,
-       two_stage_one_key_per_block, two_stage_pooled_keys]
+       two_stage_one_key_per_block, two_stage_pooled_keys, attn_matches_sdpa, attn_special_cases]

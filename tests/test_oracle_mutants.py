@@ -45,6 +45,10 @@ MUTANTS = {
                                 "int64_t kept = nbv < n_keep - 1 ? nbv : n_keep - 1;"),
     "two_stage_worst_blocks": ("c[nc++].idx = blk[j].idx * G + e;", "c[nc++].idx = blk[nbv - 1 - j].idx * G + e;"),
     "two_stage_incomplete_block": ("int64_t nbv = n / G;", "int64_t nbv = (n + G - 1) / G < nb ? (n + G - 1) / G : nb;"),
+    "attn_no_scale": ("logit[j] = scale * dot;", "logit[j] = dot;"),
+    "attn_value_from_tail": ("o[d] += e * oracle_bf16_value(vr[d]);", "o[d] += e * oracle_bf16_value(vr[Dk - Dv + d]);"),
+    "attn_not_normalised": ("for (int64_t d = 0; d < Dv; ++d) o[d] /= den;", ""),
+    "attn_padding_read": ("if (sel[j] < 0) continue;", "if (sel[j] < -1) continue;"),
 }
 
 RUNNER = r"""
