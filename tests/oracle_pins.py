@@ -245,6 +245,19 @@ def mxfp4_matches_bf16(lib):
     assert np.any(imx[:, 0] > 0)  # the keys are not all tied
 
 
+def two_stage_hand_case(lib):
+    """The two-stage case worked by hand in tests/golden/two_stage_hand.json."""
+    c = json.load(open(os.path.join(GOLDEN, "two_stage_hand.json")))
+    S, T, H, D = c["S"], c["T"], c["H"], c["D"]
+    q = _bits(np.array(c["q"], dtype=np.float32).reshape(1, S, H, D))
+    kc = _bits(np.array(c["kc"], dtype=np.float32).reshape(1, T, D))
+    w = np.array(c["w"], dtype=np.float32).reshape(1, S, H)
+    idx, sc, _ = oracle.topk_two_stage(q, kc, w, c["m"], c["k"], G=c["block"], n_keep=c["n_keep"], lib=lib)
+    want = np.array([[float(x) for x in r] for r in c["score"]], dtype=np.float32)
+    assert np.array_equal(idx, np.array(c["idx"], dtype=np.int32)), idx
+    assert np.array_equal(sc, want), sc
+
+
 def two_stage_all_kept(lib):
     """With at most n_keep complete visible blocks every visible key is a
     candidate, so the two-stage result is the one-stage top-k (rows with an
@@ -358,4 +371,5 @@ def attn_special_cases(lib):
 
 ALL = [hand_cases, onehot_matmul, positive_closed, visible_closed, causal, prefix, brute_subsets,
        invariances, batch_independent, fp8_matches_bf16, mxfp4_matches_bf16, two_stage_all_kept,
-       two_stage_one_key_per_block, two_stage_pooled_keys, attn_matches_sdpa, attn_special_cases]
+       two_stage_one_key_per_block, two_stage_pooled_keys, two_stage_hand_case, attn_matches_sdpa,
+       attn_special_cases]
