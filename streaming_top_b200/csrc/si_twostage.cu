@@ -85,6 +85,7 @@ struct FineParams {
   int* err;
   int R, T, m, G, n_keep, ldp;
   int nb;                  // complete blocks of the sequence, T / G
+  int g_shift;             // log2(G) when G is a power of two, else -1 (divide)
   long long row0;          // absolute position of chunk row 0
   uint64_t wait_limit_ns;
 };
@@ -108,13 +109,22 @@ __device__ __forceinline__ Cand cand_of(const FineParams& p, int r) {
   return c;
 }
 
+// Slot s's block within the kept list and its key within the block: shifts
+// for a power-of-two block size (the per-slot hot path), else division.
+__device__ __forceinline__ int blk_slot(const FineParams& p, int s) {
+  return p.g_shift >= 0 ? s >> p.g_shift : s / p.G;
+}
+__device__ __forceinline__ int in_blk(const FineParams& p, int s) {
+  return p.g_shift >= 0 ? s & (p.G - 1) : s % p.G;
+}
+
 // Key index of candidate slot `s` of row r, or -1 past the row's candidates
 // (and for a kept-block entry outside [0, nb), which the coarse stage never
 // writes: no address outside the keys is ever formed).
 __device__ __forceinline__ int key_of(const FineParams& p, const Cand& c, int r, int s) {
   if (s < c.n_blk_keys) {
-    const int blk = p.coarse[static_cast<long long>(r) * p.n_keep + s / p.G];
-    return blk >= 0 && blk < p.nb ? blk * p.G + s % p.G : -1;
+    const int blk = p.coarse[static_cast<long long>(r) * p.n_keep + blk_slot(p, s)];
+    return blk >= 0 && blk < p.nb ? blk * p.G + in_blk(p, s) : -1;
   }
   if (s < c.count) return c.tail0 + (s - c.n_blk_keys);
   return -1;
@@ -329,7 +339,7 @@ __global__ void __launch_bounds__(F_THREADS, 1)
         for (int j = 0; j < F_QT; ++j) {
           const int32_t* crow = p.coarse + static_cast<size_t>(U.r[j] < p.R ? U.r[j] : 0) * p.n_keep;
 #pragma unroll
-          for (int x = 0; x < 16; ++x) key[j][x] = crow[min((t * F_KT + rb + 8 * x) / p.G, p.n_keep - 1)];
+          for (int x = 0; x < 16; ++x) key[j][x] = crow[min(blk_slot(p, t * F_KT + rb + 8 * x), p.n_keep - 1)];
         }
 #pragma unroll
         for (int j = 0; j < F_QT; ++j)
@@ -338,7 +348,7 @@ __global__ void __launch_bounds__(F_THREADS, 1)
             const int s = t * F_KT + rb + 8 * x;
             const Cand& c = U.c[j];
             int kk = -1;
-            if (s < c.n_blk_keys) kk = key[j][x] >= 0 && key[j][x] < p.nb ? key[j][x] * p.G + s % p.G : -1;
+            if (s < c.n_blk_keys) kk = key[j][x] >= 0 && key[j][x] < p.nb ? key[j][x] * p.G + in_blk(p, s) : -1;
             else if (s < c.count) kk = c.tail0 + (s - c.n_blk_keys);
             key[j][x] = kk < 0 ? 0 : kk;  // an empty slot reads key 0; its score is never stored
           }
@@ -673,6 +683,7 @@ si_status launch_two_stage(const void* q, const void* kc, const float* w, int B,
       fp.n_keep = n_keep;
       fp.ldp = ldp;
       fp.nb = nb;
+      fp.g_shift = (G & (G - 1)) == 0 ? __builtin_ctz(static_cast<unsigned>(G)) : -1;
       fp.row0 = c0;
       fp.wait_limit_ns = wait_limit_ns;
       const int units = (R + F_QT - 1) / F_QT;
