@@ -245,8 +245,6 @@ def run_ours(args, wl):
     mx = args.fmt == "mxfp4"  # bf16 queries, MXFP4 keys (decoded to bf16 inside the call)
     rows_mode = args.shard == "rows"
     two = args.method == "two-stage"
-    if two and (args.fmt != "bf16" or rows_mode):
-        raise SystemExit("--method two-stage runs bf16 inputs over whole sequences")
     if rows_mode:
         # every rank holds the same sequences' keys and weights and only its
         # own query rows (equal visible pairs per rank)
@@ -483,6 +481,8 @@ def main() -> int:
                     help="N>1: independent sequences per GPU (seq, weak scaling) or the same sequences' "
                          "query rows split over the GPUs at equal visible pairs (rows, strong scaling)")
     args = ap.parse_args()
+    if args.method == "two-stage" and (args.fmt != "bf16" or args.shard == "rows"):
+        raise SystemExit("--method two-stage runs bf16 inputs over whole sequences")
     wl = synth.WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, wl)

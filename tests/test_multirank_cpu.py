@@ -173,3 +173,13 @@ def test_reference_arm_two_stage_line():
     import json
     line = json.loads(r.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["value"] > 0 and line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_bench_refuses_two_stage_with_other_formats():
+    """The two-stage bench path runs bf16 inputs over whole sequences; other
+    combinations are refused before any device work."""
+    for extra in (["--fmt", "e4m3"], ["--shard", "rows"]):
+        r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--method", "two-stage", "--workload",
+                            "tiny", "--steps", "1", "--warmup", "0", *extra],
+                           capture_output=True, text=True, timeout=300)
+        assert r.returncode != 0 and "two-stage" in (r.stderr + r.stdout), (extra, r.stderr[-300:])
