@@ -4,16 +4,21 @@ compare the CUDA path's top-k against it.
 Acceptance rules (the indexer top-k's contract):
   * integer-valued inputs: every score is exact in fp32, so indices and
     scores must match the oracle bit for bit;
-  * Gaussian inputs: the j-th returned score is within 1e-3 relative of the
-    oracle's j-th score (absolute floor 1e-6 * the row's largest score), every
-    index that is in one set but not the other has an oracle score within a
-    1e-3 relative tie window of the oracle's k-th score, and set-overlap
-    recall |G & O| / |O| has mean >= 0.9999 and min >= 0.998, where a
-    returned index whose oracle score lies within ROUND_WIN (1e-5) relative of
-    the oracle's k-th score counts as a hit: two fp32 evaluations of one
-    score differ by ~1e-7 relative, so such a key ties the k-th one within
-    rounding and which of them is kept is arbitrary.  Raw recall (no such
-    allowance) is returned too.
+  * Gaussian inputs:
+      - the j-th returned score is within 1e-3 relative of the oracle's j-th
+        score (absolute floor 1e-6 * the row's largest score);
+      - every index that is in one set but not the other has an oracle score
+        within a 1e-3 relative tie window of the oracle's k-th score;
+      - set-overlap recall |G & O| / |O| -- plain, nothing counted as a hit
+        that is not in both sets -- has mean >= 0.9999 and min >= 0.998 over
+        the compared rows.
+    A recall below that bar is a failure, with one exception that is
+    reported as an expected failure (xfail), never as a pass: every key
+    exchanged across the k-th place has an oracle score within
+    FP32_EVAL_BOUND relative of the k-th score.  That bound is the textbook
+    worst case of the fp32 evaluation of one score (a D-term dot product then
+    an H_I-term weighted sum: (D + H_I) * 2^-24 relative), so the fp32 path
+    cannot order such keys the way the fp64 oracle does.
   * always: valid entries = min(k, visible keys), -1 / -inf padding after
     them, distinct indices, every index causally visible, scores sorted
     descending.
@@ -29,8 +34,8 @@ import oracle
 import synth
 
 REL = 1e-3
-ROUND_WIN = 1e-5
 ABS_FLOOR = 1e-6
+FP32_EVAL_BOUND = (128 + 64) * 2.0 ** -24
 RECALL_MEAN = 0.9999
 RECALL_MIN = 0.998
 
@@ -113,13 +118,15 @@ def compare_exact(gi, gs, oi, osc, rows):
                            f"oracle {oi[bad[0], :8]}")
 
 
-def compare_tolerant(gi, gs, oi, osc64, rows, score_row_fn, details=None):
-    """Returns (mean recall, min recall) with rounding ties counted as hits.
+def compare_tolerant(gi, gs, oi, osc64, rows, score_row_fn) -> dict:
+    """Asserts the score tolerance and the tie window row by row, and returns
+    plain set-overlap recall: {"mean", "min", "rows", "swaps", "max_gap_rel"}.
     score_row_fn(row) -> oracle scores of all keys of that row (double), used
-    only for rows with a mismatch.  `details` (a dict) receives raw recall and
-    the largest relative gap of a mismatched key to the k-th score."""
-    recalls, raw = [], []
+    only for rows with a mismatch; "swaps" counts the keys in one set but not
+    the other, "max_gap_rel" their largest |score - k-th| / |k-th|."""
+    recalls = []
     max_gap = 0.0
+    swaps = 0
     for r in range(len(rows)):
         nv = int((oi[r] >= 0).sum())
         if nv == 0:
@@ -131,8 +138,7 @@ def compare_tolerant(gi, gs, oi, osc64, rows, score_row_fn, details=None):
         err = np.abs(g - o)
         assert np.all(err <= REL * np.abs(o) + floor), (rows[r], float(err.max()))
         G, O = set(gi[r, :nv].tolist()), set(oi[r, :nv].tolist())
-        hits = len(G & O)
-        raw.append(hits / nv)
+        recalls.append(len(G & O) / nv)
         if G != O:
             allsc = score_row_fn(int(rows[r]))
             kth = o[-1]
@@ -141,10 +147,28 @@ def compare_tolerant(gi, gs, oi, osc64, rows, score_row_fn, details=None):
                 gap = abs(allsc[x] - kth)
                 assert gap <= win, (rows[r], x, allsc[x], kth)
                 max_gap = max(max_gap, gap / max(abs(kth), 1e-30))
-            hits += sum(1 for x in G - O if abs(allsc[x] - kth) <= ROUND_WIN * abs(kth) + floor)
-        recalls.append(min(1.0, hits / nv))
+            swaps += len(G - O)
     rec = np.asarray(recalls) if recalls else np.ones(1)
-    rr = np.asarray(raw) if raw else np.ones(1)
-    if details is not None:
-        details.update(raw_mean=float(rr.mean()), raw_min=float(rr.min()), max_gap_rel=max_gap)
-    return float(rec.mean()), float(rec.min())
+    return {"mean": float(rec.mean()), "min": float(rec.min()), "rows": len(recalls),
+            "swaps": swaps, "max_gap_rel": max_gap}
+
+
+def assert_recall(*checks) -> None:
+    """checks: (stats, label) pairs from compare_tolerant.  Plain recall must
+    reach mean >= 0.9999 and min >= 0.998 in each.  A shortfall where every
+    exchanged key lies within the fp32 evaluation bound of the k-th score is
+    an expected failure (pytest.xfail with the figures, after all checks have
+    been evaluated); any other shortfall fails."""
+    soft, hard = [], []
+    for stats, what in checks:
+        if stats["mean"] >= RECALL_MEAN and stats["min"] >= RECALL_MIN:
+            continue
+        msg = (f"{what}: recall mean {stats['mean']:.6f} min {stats['min']:.6f} over {stats['rows']} rows; "
+               f"{stats['swaps']} keys exchanged at the k-th place, largest gap "
+               f"{stats['max_gap_rel']:.3g} relative to the k-th score")
+        (soft if stats["max_gap_rel"] <= FP32_EVAL_BOUND else hard).append(msg)
+    if hard:
+        raise AssertionError("; ".join(hard + soft))
+    if soft:
+        import pytest
+        pytest.xfail("; ".join(soft) + f" (all within the fp32 evaluation bound {FP32_EVAL_BOUND:.3g})")
