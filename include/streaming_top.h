@@ -27,6 +27,10 @@
  *     reported by si_device_status().
  *   - The message of the last failure on the calling host thread is available
  *     from si_last_error().
+ *   - Scratch a call needs and the caller does not pass (si_options.workspace)
+ *     is allocated and freed on `stream` from a stream-ordered memory pool the
+ *     library keeps per device; the pool holds up to 1 GiB of freed memory
+ *     between calls so that repeated calls do not map memory anew.
  */
 #ifndef STREAMING_TOP_H
 #define STREAMING_TOP_H
@@ -83,6 +87,12 @@ typedef struct si_options {
                             2^(byte-127) (device).  The keys are decoded to bf16 (exact for scales
                             <= 252) into B*T*D*2 bytes of scratch -- opt->workspace when given,
                             else allocated and freed on `stream` -- then scored as bf16. */
+  int32_t* device_status;  /* optional: this call's own device error word, int32_t[2] in device
+                            memory, 8-byte aligned, zeroed by the caller.  A kernel of the call
+                            whose bounded wait runs out writes SI_ERR_TIMEOUT into [0] and the
+                            waiting site into [1] (the first failure wins) and exits early.  NULL
+                            (default): the library's per-device record, which si_device_status()
+                            reads and clears, is used instead. */
 } si_options;
 
 /*
@@ -121,6 +131,39 @@ SI_API si_status si_indexer_topk_rows(const void* q, const void* kc, const float
                                       float* out_score, void* stream, const si_options* opt);
 
 /*
+ * Streaming indexer top-k on HOST buffers, end to end: rows row0 .. row0+R-1
+ * of every sequence, laid out as si_indexer_topk_rows's arguments but in
+ * host memory: q [B,R,H_I,D], w [B,R,H_I], kc [B,T,D] (all T keys), results
+ * out_idx / out_score [B,R,k] (out_score may be NULL); for fp8, opt->q_scale
+ * [B,R,H_I] and opt->kc_scale [B,T] are host pointers too, and for MXFP4
+ * keys opt->kc_mx_scale [B,T,D/32].  row0 = 0, R = S is the whole sequence.
+ * The pages stream the queries in chunks so that only one chunk is resident
+ * (StreamIndex abstract, the memory bound at a million tokens); this call
+ * does so from host memory: the keys are copied once, then chunks of
+ * opt->query_chunk rows (0 = 8192; a multiple of 4) go through two device
+ * slots, the copy of the next chunk in and of the previous chunk's results
+ * out overlapping the scoring of the current one (two internal copy streams
+ * ordered against `stream` by events).  Device memory: the keys plus two
+ * chunks of q, w and results, si_indexer_topk_host_workspace_size() bytes,
+ * from opt->workspace when given, else allocated and freed on `stream`.
+ * Host buffers must stay valid for the call; page-locked memory
+ * (cudaHostAlloc / cudaHostRegister) is needed for the copies to overlap,
+ * pageable memory works but copies synchronously.  Blocks until the results
+ * are in the host buffers.  Returns what si_indexer_topk_rows would, or
+ * SI_ERR_TIMEOUT when a kernel's bounded wait ran out (read from
+ * opt->device_status when given, else from the device record as
+ * si_device_status() does).
+ */
+SI_API si_status si_indexer_topk_host(const void* q, const void* kc, const float* w, int B, int row0, int R,
+                                      int T, int H_I, int D, int m, int k, int32_t* out_idx, float* out_score,
+                                      void* stream, const si_options* opt);
+
+/* Device bytes si_indexer_topk_host needs for these arguments (its
+ * opt->query_chunk and dtype; with_score != 0 when out_score is given). */
+SI_API size_t si_indexer_topk_host_workspace_size(int B, int R, int T, int H_I, int D, int k, int with_score,
+                                                  const si_options* opt);
+
+/*
  * Sorts every row of a top-k result in place by (score descending, index
  * ascending): idx [rows, k] int32, score [rows, k] fp32, device memory, one
  * row per query.  Entries with index -1 and score -inf (padding) end up last.
@@ -151,15 +194,19 @@ SI_API si_status si_indexer_materialize(const void* q, const void* kc, const flo
  * latency-critical loop where cudaMalloc/cudaFree would synchronise).  It has
  * no counterpart on the pages: it runs the same materialize kernels with
  * their scratch in a fixed device array of SI_NOALLOC_SCRATCH_BYTES that the
- * library holds on every GPU that loads it, until the process exits.
+ * library holds on every GPU where its module is loaded, until the process
+ * exits.  Under CUDA's lazy module loading (the default) the array is
+ * reserved by the first call on each device, which therefore needs that
+ * much free memory itself (SI_ERR_OUT_OF_MEMORY if not): make that first
+ * call, on a small problem, before the caller's own pool takes the memory.
  *   Same arguments, layouts, ownership and results as
  *   si_indexer_materialize (bf16 q, kc; fp32 w; device pointers).
  *   Returns SI_ERR_UNSUPPORTED, touching nothing, when the scratch need
  *   4*B*S*T*(H_I+1) + 256 bytes exceeds SI_NOALLOC_SCRATCH_BYTES, or T >
  *   16384.  Calls no cudaMalloc / cudaFree and nothing that allocates.
- *   The first call on a device looks up the array's device address (once per
- *   device, with that device current); make that first call before any
- *   stream capture.
+ *   Every call looks up the array's device address in the current context
+ *   (cudaGetSymbolAddress, which allocates nothing once the module is
+ *   loaded); make the first call on a device before any stream capture.
  *   All calls on a device share the array, which keeps the last call's
  *   contents (every word is overwritten before it is read); calls whose
  *   work overlaps on the same device race on it and must be serialised.
@@ -202,6 +249,29 @@ SI_API si_status si_indexer_topk_two_stage(const void* q, const void* kc, const 
 SI_API size_t si_two_stage_workspace_size(int B, int S, int T, int block, int n_keep, int query_chunk);
 
 /*
+ * Sparse attention over the selected compressed latents: the consumer of the
+ * top-k (StreamIndex abstract: the sparse attention kernel reads only the
+ * entries the indexer selected).  Reading of the pages (the DeepSeek-V3.2
+ * lineage the V4.1 page gives): each of the H heads of query t attends over
+ * the k latents idx[b,t,:] of its sequence (index -1 is padding and is
+ * skipped); a latent serves as the key (all Dk values) and as the value (its
+ * first Dv values); the softmax runs over the selection only, with `scale`
+ * (0 = 1/sqrt(Dk)).
+ *   q   [B, S, H, Dk] bf16     kv  [B, T, Dk] bf16     idx [B, S, k] int32
+ *   out [B, S, H, Dv] bf16 (written): sum_j softmax_j(scale q.kv_j) kv_j[:Dv]
+ *   lse [B, S, H] fp32 (written): ln sum_j exp(scale q.kv_j)
+ * A row with nothing selected gives out = 0 and lse = -inf.  Supported:
+ * H == 64, Dk == 576, Dv == 512, k in {128, 256, 384, 512}; entries of idx
+ * outside [-1, T) are treated as padding.  The softmax weights are rounded to
+ * bf16 for the value product (their rounded sum normalises it).  Device
+ * pointers, 16-byte aligned; asynchronous on `stream`; opt may be NULL (its
+ * device_status is honoured, the other fields are ignored).
+ */
+SI_API si_status si_sparse_attention(const void* q, const void* kv, const int32_t* idx, int B, int S, int T,
+                                     int H, int Dk, int Dv, int k, float scale, void* out, float* lse,
+                                     void* stream, const si_options* opt);
+
+/*
  * Decodes MXFP4 rows to bf16: codes [rows, D/2] bytes (value d in the low
  * nibble of byte d/2 when d is even, the high nibble when odd), E8M0 scales
  * [rows, D/32] (one per 32 values), out [rows, D] bf16; device pointers,
@@ -214,15 +284,20 @@ SI_API size_t si_two_stage_workspace_size(int B, int S, int T, int block, int n_
 SI_API si_status si_mxfp4_to_bf16(const void* codes, const void* scales, int64_t rows, int D, void* out,
                                   void* stream);
 
-/* Scratch bytes a call with these arguments needs (0 if none).  materialize
- * selects the materialize path's need; otherwise the streaming path's, which
- * is B*T*D*2 (+ alignment) for SI_DTYPE_MXFP4_KEYS and 0 for the others. */
+/* Scratch bytes a call with these arguments needs (0 if none).  One function
+ * serves two entry points, so it takes one argument more than the call it
+ * sizes: materialize != 0 gives si_indexer_materialize's need,
+ * 4*B*S*T*(H_I+1) + 256; materialize == 0 the streaming path's, which is
+ * B*T*D*2 (+ alignment) for SI_DTYPE_MXFP4_KEYS and 0 for the others. */
 SI_API size_t si_indexer_workspace_size(int B, int S, int T, int H_I, int D, int m, int k, int materialize,
                                  const si_options* opt);
 
 /* Waits for `stream`, then returns SI_ERR_TIMEOUT (and clears the record) if
- * any kernel of this library timed out in a bounded wait since the last call,
- * else the stream's own error state (SI_OK or SI_ERR_CUDA). */
+ * any kernel of this library that ran without its own si_options.device_status
+ * word timed out in a bounded wait since the last call, else the stream's own
+ * error state (SI_OK or SI_ERR_CUDA).  The record is per device and shared by
+ * every stream and host thread on it; a caller that needs a per-call status
+ * passes si_options.device_status instead. */
 SI_API si_status si_device_status(void* stream);
 
 SI_API const char* si_status_string(si_status s);

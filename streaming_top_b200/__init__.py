@@ -36,7 +36,7 @@ _vp, _i, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
 class Options(ctypes.Structure):
     _fields_ = [("dtype", _i), ("q_scale", _vp), ("kc_scale", _vp), ("query_chunk", _i),
                 ("key_tile", _i), ("workspace", _vp), ("workspace_bytes", _sz), ("unsorted", _i),
-                ("kc_mx_scale", _vp)]
+                ("kc_mx_scale", _vp), ("device_status", _vp)]
 
 
 _ARGS = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp]
@@ -47,6 +47,11 @@ _lib.si_indexer_topk_ex.argtypes = _ARGS + [ctypes.POINTER(Options)]
 _lib.si_indexer_topk_rows.restype = _i
 _lib.si_indexer_topk_rows.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp,
                                       ctypes.POINTER(Options)]
+_lib.si_indexer_topk_host.restype = _i
+_lib.si_indexer_topk_host.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp,
+                                      ctypes.POINTER(Options)]
+_lib.si_indexer_topk_host_workspace_size.restype = _sz
+_lib.si_indexer_topk_host_workspace_size.argtypes = [_i] * 7 + [ctypes.POINTER(Options)]
 _lib.si_sort_topk_rows.restype = _i
 _lib.si_sort_topk_rows.argtypes = [_vp, _vp, ctypes.c_int64, _i, _vp]
 _lib.si_indexer_materialize.restype = _i
@@ -60,6 +65,9 @@ _lib.si_indexer_topk_two_stage.restype = _i
 _lib.si_indexer_topk_two_stage.argtypes = [_vp, _vp, _vp] + [_i] * 9 + [_vp, _vp, _vp, ctypes.POINTER(Options)]
 _lib.si_two_stage_workspace_size.restype = _sz
 _lib.si_two_stage_workspace_size.argtypes = [_i] * 6
+_lib.si_sparse_attention.restype = _i
+_lib.si_sparse_attention.argtypes = [_vp, _vp, _vp] + [_i] * 7 + [ctypes.c_float, _vp, _vp, _vp,
+                                                                    ctypes.POINTER(Options)]
 _lib.si_mxfp4_to_bf16.restype = _i
 _lib.si_mxfp4_to_bf16.argtypes = [_vp, _vp, ctypes.c_int64, _i, _vp, _vp]
 _lib.si_device_status.restype = _i
@@ -69,8 +77,11 @@ _lib.si_status_string.argtypes = [_i]
 _lib.si_last_error.restype = ctypes.c_char_p
 _lib.si_last_error.argtypes = []
 _lib.si_version.restype = _i
+_lib.si_version.argtypes = []
+_lib.si_test_fail_allocations.restype = None
+_lib.si_test_fail_allocations.argtypes = [_i]
 _lib.si_test_stream_timeout.restype = _i
-_lib.si_test_stream_timeout.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, ctypes.c_ulonglong]
+_lib.si_test_stream_timeout.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, ctypes.c_ulonglong, _vp]
 
 
 class SIError(RuntimeError):
@@ -99,7 +110,7 @@ def _stream_ptr(stream) -> int:
     return s.cuda_stream
 
 
-def _shapes(q, kc, w, mxfp4: bool = False):
+def _shapes(q, kc, w, mxfp4: bool = False, host: bool = False):
     if q.dim() != 4 or kc.dim() != 3 or w.dim() != 3:
         raise ValueError("q [B,S,H,D], kc [B,T,D] (MXFP4: [B,T,D/2] codes), w [B,S,H] expected")
     B, S, H, D = q.shape
@@ -107,8 +118,8 @@ def _shapes(q, kc, w, mxfp4: bool = False):
     if kc.shape[0] != B or kc.shape[2] != kd or tuple(w.shape) != (B, S, H):
         raise ValueError(f"shape mismatch q{tuple(q.shape)} kc{tuple(kc.shape)} w{tuple(w.shape)}")
     for name, t in (("q", q), ("kc", kc), ("w", w)):
-        if not t.is_cuda or not t.is_contiguous():
-            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+        if t.is_cuda == host or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous {'host (CPU)' if host else 'CUDA'} tensor")
     if w.dtype != torch.float32:
         raise ValueError("w must be float32")
     return B, S, kc.shape[1], H, D
@@ -122,8 +133,14 @@ def _outputs(B, S, k, device, out_idx, out_score, with_score):
     return out_idx, out_score
 
 
-def _options(q, kc, q_scale, kc_scale, query_chunk, key_tile, workspace=None, kc_mx_scale=None):
+def _options(q, kc, q_scale, kc_scale, query_chunk, key_tile, workspace=None, kc_mx_scale=None,
+             device_status=None):
     o = Options()
+    if device_status is not None:
+        if (device_status.dtype != torch.int32 or device_status.numel() < 2 or not device_status.is_cuda
+                or not device_status.is_contiguous()):
+            raise ValueError("device_status must be a contiguous int32 CUDA tensor of >= 2 elements")
+        o.device_status = device_status.data_ptr()
     if kc_mx_scale is not None:
         B, _, _, D = q.shape
         shape = (B, kc.shape[1], D // 32)
@@ -161,14 +178,16 @@ def _options(q, kc, q_scale, kc_scale, query_chunk, key_tile, workspace=None, kc
 
 def indexer_topk(q, kc, w, m: int, k: int, *, q_scale=None, kc_scale=None, query_chunk: int = 0,
                  key_tile: int = 0, out_idx=None, out_score=None, with_score: bool = True,
-                 unsorted: bool = False, stream=None, kc_mx_scale=None, workspace=None):
+                 unsorted: bool = False, stream=None, kc_mx_scale=None, workspace=None, device_status=None):
     """Streaming indexer top-k (``si_indexer_topk_ex``).  Returns (idx, score).
     With unsorted=True each row's results come in an unspecified order (valid
     entries first) and the row sort is skipped.  With kc_mx_scale (uint8
-    [B,T,D/32] E8M0), kc holds MXFP4 codes [B,T,D/2] (uint8) and q is bf16."""
+    [B,T,D/32] E8M0), kc holds MXFP4 codes [B,T,D/2] (uint8) and q is bf16.
+    device_status: optional zeroed int32 CUDA tensor (>= 2 elements), this
+    call's own device error word."""
     B, S, T, H, D = _shapes(q, kc, w, kc_mx_scale is not None)
     out_idx, out_score = _outputs(B, S, k, q.device, out_idx, out_score, with_score)
-    o = _options(q, kc, q_scale, kc_scale, query_chunk, key_tile, workspace, kc_mx_scale)
+    o = _options(q, kc, q_scale, kc_scale, query_chunk, key_tile, workspace, kc_mx_scale, device_status)
     o.unsorted = int(bool(unsorted))
     st = _lib.si_indexer_topk_ex(q.data_ptr(), kc.data_ptr(), w.data_ptr(), B, S, T, H, D, m, k,
                                  out_idx.data_ptr(), out_score.data_ptr() if out_score is not None else None,
@@ -180,13 +199,13 @@ def indexer_topk(q, kc, w, m: int, k: int, *, q_scale=None, kc_scale=None, query
 def indexer_topk_rows(q, kc, w, m: int, k: int, row0: int, *, q_scale=None, kc_scale=None,
                       query_chunk: int = 0, key_tile: int = 0, out_idx=None, out_score=None,
                       with_score: bool = True, unsorted: bool = False, stream=None, kc_mx_scale=None,
-                      workspace=None):
+                      workspace=None, device_status=None):
     """Streaming top-k for query rows row0 .. row0+R-1 (``si_indexer_topk_rows``):
     q [B, R, H_I, D] and w [B, R, H_I] hold those rows only, kc [B, T, D] all
     keys.  Returns (idx, score) of shape [B, R, k]."""
     B, R, T, H, D = _shapes(q, kc, w, kc_mx_scale is not None)
     out_idx, out_score = _outputs(B, R, k, q.device, out_idx, out_score, with_score)
-    o = _options(q, kc, q_scale, kc_scale, query_chunk, key_tile, workspace, kc_mx_scale)
+    o = _options(q, kc, q_scale, kc_scale, query_chunk, key_tile, workspace, kc_mx_scale, device_status)
     o.unsorted = int(bool(unsorted))
     st = _lib.si_indexer_topk_rows(q.data_ptr(), kc.data_ptr(), w.data_ptr(), B, int(row0), R, T, H, D,
                                    m, k, out_idx.data_ptr(),
@@ -197,14 +216,15 @@ def indexer_topk_rows(q, kc, w, m: int, k: int, row0: int, *, q_scale=None, kc_s
 
 
 def indexer_topk_two_stage(q, kc, w, m: int, k: int, *, block: int = 8, n_keep: int = 2048,
-                           query_chunk: int = 0, out_idx=None, out_score=None, workspace=None, stream=None):
+                           query_chunk: int = 0, out_idx=None, out_score=None, workspace=None, stream=None,
+                           device_status=None):
     """Two-stage indexer top-k (``si_indexer_topk_two_stage``): the best
     n_keep blocks of `block` keys by the score of their pooled (mean) key,
     then the top-k of their keys and the incomplete block's visible keys.
     Returns (idx, score) [B, S, k], ordered as indexer_topk's."""
     B, S, T, H, D = _shapes(q, kc, w)
     out_idx, out_score = _outputs(B, S, k, q.device, out_idx, out_score, True)
-    o = _options(q, kc, None, None, query_chunk, 0, workspace)
+    o = _options(q, kc, None, None, query_chunk, 0, workspace, device_status=device_status)
     st = _lib.si_indexer_topk_two_stage(q.data_ptr(), kc.data_ptr(), w.data_ptr(), B, S, T, H, D, m, k,
                                         int(block), int(n_keep), out_idx.data_ptr(), out_score.data_ptr(),
                                         _stream_ptr(stream), ctypes.byref(o))
@@ -214,6 +234,33 @@ def indexer_topk_two_stage(q, kc, w, m: int, k: int, *, block: int = 8, n_keep: 
 
 def two_stage_workspace_size(B, S, T, block=8, n_keep=2048, query_chunk=0) -> int:
     return int(_lib.si_two_stage_workspace_size(B, S, T, block, n_keep, query_chunk))
+
+
+def sparse_attention(q, kv, idx, *, scale: float = 0.0, out=None, lse=None, stream=None, device_status=None):
+    """Sparse attention over the selected latents (``si_sparse_attention``):
+    q [B,S,H,Dk] bf16, kv [B,T,Dk] bf16, idx [B,S,k] int32 (-1 padding).
+    Returns (out [B,S,H,Dv=512] bf16, lse [B,S,H] fp32)."""
+    if q.dim() != 4 or kv.dim() != 3 or idx.dim() != 3:
+        raise ValueError("q [B,S,H,Dk], kv [B,T,Dk], idx [B,S,k] expected")
+    B, S, H, Dk = q.shape
+    T, k = kv.shape[1], idx.shape[2]
+    Dv = 512
+    if kv.shape[0] != B or kv.shape[2] != Dk or idx.shape[:2] != (B, S):
+        raise ValueError(f"shape mismatch q{tuple(q.shape)} kv{tuple(kv.shape)} idx{tuple(idx.shape)}")
+    for name, t, dt in (("q", q, torch.bfloat16), ("kv", kv, torch.bfloat16), ("idx", idx, torch.int32)):
+        if not t.is_cuda or not t.is_contiguous() or t.dtype != dt:
+            raise ValueError(f"{name} must be a contiguous {dt} CUDA tensor")
+    if out is None:
+        out = torch.empty((B, S, H, Dv), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, S, H), dtype=torch.float32, device=q.device)
+    o = Options()
+    if device_status is not None:
+        o.device_status = device_status.data_ptr()
+    _check(_lib.si_sparse_attention(q.data_ptr(), kv.data_ptr(), idx.data_ptr(), B, S, T, H, Dk, Dv, k,
+                                    float(scale), out.data_ptr(), lse.data_ptr(), _stream_ptr(stream),
+                                    ctypes.byref(o)), "si_sparse_attention")
+    return out, lse
 
 
 def mxfp4_to_bf16(codes, scales, out=None, stream=None):
@@ -280,8 +327,12 @@ def indexer_materialize_noalloc(q, kc, w, m: int, k: int, *, out_idx=None, out_s
     return out_idx, out_score
 
 
-def workspace_size(B, S, T, H, D, m, k, materialize: bool = False) -> int:
-    return int(_lib.si_indexer_workspace_size(B, S, T, H, D, m, k, int(materialize), None))
+def workspace_size(B, S, T, H, D, m, k, materialize: bool = False, mxfp4: bool = False) -> int:
+    """si_indexer_workspace_size: the materialize path's scratch, or the
+    streaming path's (the decoded keys for MXFP4 keys, else 0)."""
+    o = Options()
+    o.dtype = SI_DTYPE_MXFP4_KEYS if mxfp4 else SI_DTYPE_BF16
+    return int(_lib.si_indexer_workspace_size(B, S, T, H, D, m, k, int(materialize), ctypes.byref(o)))
 
 
 def device_status(stream=None) -> int:
@@ -289,17 +340,87 @@ def device_status(stream=None) -> int:
     return int(_lib.si_device_status(_stream_ptr(stream)))
 
 
-def indexer_topk_host(q, kc, w, m: int, k: int, *, q_scale=None, kc_scale=None, device="cuda",
-                      query_chunk: int = 0, key_tile: int = 0, bufs: dict | None = None,
-                      sync: bool = True, row0: int | None = None, kc_mx_scale=None,
-                      two_stage: dict | None = None):
-    """End-to-end call on HOST tensors (pinned for best speed): copies the
-    inputs to the device, runs the streaming top-k, copies (idx, score) back.
-    `bufs` may hold reusable device buffers from a previous call.  With
-    sync=False the copies back are only enqueued on the current stream.
-    With `row0`, q and w hold only rows row0 .. row0+R-1 of the sequences
-    (si_indexer_topk_rows).  With `two_stage` (keyword arguments of
-    indexer_topk_two_stage: block, n_keep), the two-stage indexer runs."""
+def _host_options(q, kc, q_scale, kc_scale, kc_mx_scale, query_chunk, key_tile, unsorted, device_status):
+    """si_options for the host-buffer entry point: the scales are host tensors."""
+    o = Options()
+    if kc_mx_scale is not None:
+        if q.dtype != torch.bfloat16 or kc.dtype != torch.uint8 or kc_mx_scale.dtype != torch.uint8:
+            raise ValueError("MXFP4 keys: q bfloat16, kc uint8 codes and kc_mx_scale uint8 expected")
+        o.dtype = SI_DTYPE_MXFP4_KEYS
+        o.kc_mx_scale = kc_mx_scale.data_ptr()
+    elif q.dtype == torch.bfloat16 and kc.dtype == torch.bfloat16:
+        o.dtype = SI_DTYPE_BF16
+    elif q.dtype in (torch.uint8, torch.float8_e4m3fn) and kc.element_size() == 1:
+        if q_scale is None or kc_scale is None:
+            raise ValueError("fp8 inputs need q_scale and kc_scale")
+        o.dtype = SI_DTYPE_FP8_E4M3
+        o.q_scale = q_scale.data_ptr()
+        o.kc_scale = kc_scale.data_ptr()
+    else:
+        raise ValueError(f"unsupported q / kc dtypes {q.dtype} / {kc.dtype}")
+    for name, t in (("q", q), ("kc", kc), ("q_scale", q_scale), ("kc_scale", kc_scale),
+                    ("kc_mx_scale", kc_mx_scale)):
+        if t is not None and (t.is_cuda or not t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous host (CPU) tensor")
+    o.query_chunk = int(query_chunk)
+    o.key_tile = int(key_tile)
+    o.unsorted = int(bool(unsorted))
+    if device_status is not None:
+        o.device_status = device_status.data_ptr()
+    return o
+
+
+def indexer_topk_host(q, kc, w, m: int, k: int, *, q_scale=None, kc_scale=None, row0: int | None = None,
+                      query_chunk: int = 0, key_tile: int = 0, out_idx=None, out_score=None,
+                      with_score: bool = True, unsorted: bool = False, stream=None, kc_mx_scale=None,
+                      device_status=None, device=None, workspace=None):
+    """End to end on HOST tensors (``si_indexer_topk_host``): q [B, R, H_I, D],
+    w [B, R, H_I], kc [B, T, D] (and the fp8 / MXFP4 scales) in host memory,
+    page-locked for the copies to overlap the scoring.  The library copies the
+    keys once and the query rows in chunks of `query_chunk` rows (0 = 8192)
+    through two device slots, overlapping the copies with the scoring, and
+    returns when (idx, score) [B, R, k] are in host memory.  With `row0` the
+    rows are rows row0 .. row0+R-1 of the sequences (default 0: the whole
+    sequence).  `device` selects the GPU (default: the current one);
+    `workspace` (a CUDA uint8 tensor of indexer_topk_host_workspace_size()
+    bytes) replaces the call's own device allocation."""
+    B, R, T, H, D = _shapes(q, kc, w, kc_mx_scale is not None, host=True)
+    pin = q.is_pinned()
+    if out_idx is None:
+        out_idx = torch.empty((B, R, k), dtype=torch.int32, pin_memory=pin)
+    if out_score is None and with_score:
+        out_score = torch.empty((B, R, k), dtype=torch.float32, pin_memory=pin)
+    for name, t in (("out_idx", out_idx), ("out_score", out_score)):
+        if t is not None and (t.is_cuda or not t.is_contiguous() or tuple(t.shape) != (B, R, k)):
+            raise ValueError(f"{name} must be a contiguous host tensor of shape {(B, R, k)}")
+    o = _host_options(q, kc, q_scale, kc_scale, kc_mx_scale, query_chunk, key_tile, unsorted, device_status)
+    if workspace is not None:
+        if not workspace.is_cuda or not workspace.is_contiguous():
+            raise ValueError("workspace must be a contiguous CUDA tensor")
+        o.workspace = workspace.data_ptr()
+        o.workspace_bytes = workspace.numel() * workspace.element_size()
+    with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
+        st = _lib.si_indexer_topk_host(q.data_ptr(), kc.data_ptr(), w.data_ptr(), B, int(row0 or 0), R, T, H, D,
+                                       m, k, out_idx.data_ptr(),
+                                       out_score.data_ptr() if out_score is not None else None,
+                                       _stream_ptr(stream), ctypes.byref(o))
+    _check(st, "si_indexer_topk_host")
+    return out_idx, out_score
+
+
+def indexer_topk_host_workspace_size(B, R, T, H, D, k, *, with_score=True, query_chunk=0, dtype=SI_DTYPE_BF16):
+    o = Options()
+    o.dtype = dtype
+    o.query_chunk = int(query_chunk)
+    return int(_lib.si_indexer_topk_host_workspace_size(B, R, T, H, D, k, int(with_score), ctypes.byref(o)))
+
+
+def indexer_topk_two_stage_host(q, kc, w, m: int, k: int, *, device="cuda", query_chunk: int = 0,
+                                bufs: dict | None = None, sync: bool = True, **two_stage):
+    """The two-stage indexer end to end on HOST tensors: copies q, kc and w
+    to the device, runs ``si_indexer_topk_two_stage`` and copies (idx, score)
+    back.  `bufs` may hold reusable device buffers from a previous call; with
+    sync=False the copies back are only enqueued on the current stream."""
     bufs = {} if bufs is None else bufs
     stream = torch.cuda.current_stream(device)
 
@@ -312,24 +433,19 @@ def indexer_topk_host(q, kc, w, m: int, k: int, *, q_scale=None, kc_scale=None, 
         return d
 
     qd, kd, wd = dev("q", q), dev("kc", kc), dev("w", w)
-    qs = dev("q_scale", q_scale) if q_scale is not None else None
-    ks = dev("kc_scale", kc_scale) if kc_scale is not None else None
-    kms = dev("kc_mx_scale", kc_mx_scale) if kc_mx_scale is not None else None
     B, S = q.shape[0], q.shape[1]
     oi = bufs.get("out_idx")
     os_ = bufs.get("out_score")
     if oi is None or oi.shape != (B, S, k):
         oi = bufs["out_idx"] = torch.empty((B, S, k), dtype=torch.int32, device=device)
         os_ = bufs["out_score"] = torch.empty((B, S, k), dtype=torch.float32, device=device)
-    if two_stage is not None:
-        indexer_topk_two_stage(qd, kd, wd, m, k, query_chunk=query_chunk, out_idx=oi, out_score=os_,
-                               stream=stream, **two_stage)
-    elif row0 is None:
-        indexer_topk(qd, kd, wd, m, k, q_scale=qs, kc_scale=ks, query_chunk=query_chunk,
-                     key_tile=key_tile, out_idx=oi, out_score=os_, stream=stream, kc_mx_scale=kms)
-    else:
-        indexer_topk_rows(qd, kd, wd, m, k, row0, q_scale=qs, kc_scale=ks, query_chunk=query_chunk,
-                          key_tile=key_tile, out_idx=oi, out_score=os_, stream=stream, kc_mx_scale=kms)
+    ws = bufs.get("workspace")
+    need = two_stage_workspace_size(B, S, kc.shape[1], two_stage.get("block", 8), two_stage.get("n_keep", 2048),
+                                    query_chunk)
+    if ws is None or ws.numel() < need:
+        ws = bufs["workspace"] = torch.empty(need, dtype=torch.uint8, device=device)
+    indexer_topk_two_stage(qd, kd, wd, m, k, query_chunk=query_chunk, out_idx=oi, out_score=os_,
+                           stream=stream, workspace=ws, **two_stage)
     hi = bufs.get("h_idx")
     hs = bufs.get("h_score")
     if hi is None or hi.shape != oi.shape:
@@ -379,10 +495,23 @@ def row_shards(S: int, T: int, m: int, parts: int, align: int = 4) -> list[int]:
     return bounds
 
 
-def test_stream_timeout(q, kc, w, m: int, k: int, out_idx, wait_limit_ns: int, stream=None) -> int:
+def test_stream_timeout(q, kc, w, m: int, k: int, out_idx, wait_limit_ns: int, stream=None,
+                        device_status=None) -> int:
     """Test hook: run the streaming kernel with one key tile withheld and a
-    short bounded-wait limit; returns the launch status (the timeout itself is
-    reported by device_status())."""
+    short bounded-wait limit; returns the launch status.  The timeout itself
+    lands in device_status (a zeroed int32 CUDA tensor of >= 2 elements) when
+    given, else in the record device_status() reads."""
     B, S, T, H, D = _shapes(q, kc, w)
+    ds = None
+    if device_status is not None:
+        if device_status.dtype != torch.int32 or device_status.numel() < 2 or not device_status.is_cuda:
+            raise ValueError("device_status must be an int32 CUDA tensor of >= 2 elements")
+        ds = device_status.data_ptr()
     return int(_lib.si_test_stream_timeout(q.data_ptr(), kc.data_ptr(), w.data_ptr(), B, S, T, m, k,
-                                           out_idx.data_ptr(), _stream_ptr(stream), wait_limit_ns))
+                                           out_idx.data_ptr(), _stream_ptr(stream), wait_limit_ns, ds))
+
+
+def test_fail_allocations(n: int) -> None:
+    """Test hook: the library's next n scratch allocations fail as if the
+    device were out of memory (``si_test_fail_allocations``)."""
+    _lib.si_test_fail_allocations(int(n))

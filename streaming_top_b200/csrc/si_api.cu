@@ -3,6 +3,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -18,9 +20,41 @@ thread_local char g_last_error[512] = "";
 // Error record written by the kernels of this library (per device).
 __device__ int g_device_error[4];
 
+// Test hook: the next g_fail_allocs scratch allocations of the library fail.
+std::atomic<int> g_fail_allocs{0};
+
+// The library's stream-ordered memory pool per device.  Scratch that calls
+// allocate and free on their stream comes from it; it keeps up to
+// kPoolKeepBytes of freed memory between calls (the default pool would give
+// it back at every synchronisation and make the next call map it anew).
 constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-int* g_err_ptr[kMaxDevices] = {};
+constexpr uint64_t kPoolKeepBytes = 1ull << 30;
+std::mutex g_pool_mu;
+cudaMemPool_t g_pool[kMaxDevices] = {};
+
+cudaError_t library_pool(int dev, bool renew, cudaMemPool_t* out) {
+  std::lock_guard<std::mutex> lk(g_pool_mu);
+  if (renew && g_pool[dev]) g_pool[dev] = nullptr;  // a device reset destroyed it: make another
+  if (!g_pool[dev]) {
+    cudaMemPoolProps props;
+    std::memset(&props, 0, sizeof props);
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pool = nullptr;
+    cudaError_t e = cudaMemPoolCreate(&pool, &props);
+    if (e != cudaSuccess) return e;
+    uint64_t keep = kPoolKeepBytes;
+    e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+    if (e != cudaSuccess) {
+      cudaMemPoolDestroy(pool);
+      return e;
+    }
+    g_pool[dev] = pool;
+  }
+  *out = g_pool[dev];
+  return cudaSuccess;
+}
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -48,20 +82,48 @@ si_status cuda_fail(cudaError_t e, const char* what) {
   return fail(SI_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
 }
 
+// The record's address in the current context, asked for on every call (no
+// cache that a device reset or another context could make stale).
 si_status device_error_record(int** out) {
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_device_error);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(error record)");
+  *out = static_cast<int*>(p);
+  return SI_OK;
+}
+
+si_status error_word(const si_options* opt, int** out) {
+  if (opt && opt->device_status) {
+    if (reinterpret_cast<uintptr_t>(opt->device_status) % 8 != 0)
+      return fail(SI_ERR_INVALID_ARGUMENT, "device_status must be 8-byte aligned");
+    *out = opt->device_status;
+    return SI_OK;
+  }
+  return device_error_record(out);
+}
+
+si_status scratch_alloc(void** p, size_t bytes, cudaStream_t stream, const char* what) {
+  *p = nullptr;
+  int left = g_fail_allocs.load();
+  while (left > 0 && !g_fail_allocs.compare_exchange_weak(left, left - 1)) {
+  }
+  if (left > 0)
+    return fail(SI_ERR_OUT_OF_MEMORY, "allocating %zu bytes for %s: failed by the allocation-failure test hook",
+                bytes, what);
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   if (dev < 0 || dev >= kMaxDevices) return fail(SI_ERR_UNSUPPORTED, "device index %d", dev);
-  std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_err_ptr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_device_error);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(error record)");
-    g_err_ptr[dev] = static_cast<int*>(p);
+  for (int attempt = 0; attempt < 2; ++attempt) {
+    cudaMemPool_t pool = nullptr;
+    e = library_pool(dev, attempt > 0, &pool);
+    if (e == cudaSuccess) e = cudaMallocFromPoolAsync(p, bytes, pool, stream);
+    if (e == cudaSuccess) return SI_OK;
+    cudaGetLastError();
+    *p = nullptr;
+    if (e == cudaErrorMemoryAllocation) break;
   }
-  *out = g_err_ptr[dev];
-  return SI_OK;
+  return fail(SI_ERR_OUT_OF_MEMORY, "cudaMallocFromPoolAsync(%zu) for %s: %s", bytes, what, cudaGetErrorString(e));
 }
 
 si_status encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
@@ -101,9 +163,7 @@ si_status check_common(const void* q, const void* kc, const float* w, int B, int
 
 }  // namespace si
 
-using namespace si;
-
-namespace {
+namespace si {
 
 // Scratch for MXFP4 keys decoded to bf16: [B, T, D] bf16 plus alignment slack.
 size_t mxfp4_key_bytes(int B, int T, int D) {
@@ -162,6 +222,18 @@ si_status stream_topk_rows(const void* q, const void* kc, const float* w, int B,
   cfg.test_withhold = 0;
   cfg.unsorted = o.unsorted != 0;
   cfg.row0 = row0;
+  st = error_word(&o, &cfg.err);
+  if (st != SI_OK) return st;
+  bool sorted_by_merge = false;
+  cfg.out_sorted = &sorted_by_merge;
+  // the caller's workspace: the decoded MXFP4 keys first, then the split-key partials
+  if (o.workspace) {
+    const size_t used = mx ? mxfp4_key_bytes(B, T, D) : 0;
+    if (o.workspace_bytes > used) {
+      cfg.split_ws = static_cast<uint8_t*>(o.workspace) + used;
+      cfg.split_ws_bytes = o.workspace_bytes - used;
+    }
+  }
   const cudaStream_t cs = static_cast<cudaStream_t>(stream);
   // MXFP4 keys: decode them to bf16 scratch first (exact), then score as bf16
   void* kraw = nullptr;  // the allocation, when the library made it
@@ -169,12 +241,8 @@ si_status stream_topk_rows(const void* q, const void* kc, const float* w, int B,
     const size_t need = mxfp4_key_bytes(B, T, D);
     void* base = o.workspace;
     if (!base) {
-      cudaError_t e = cudaMallocAsync(&kraw, need, cs);
-      if (e != cudaSuccess) {
-        cudaGetLastError();
-        return fail(SI_ERR_OUT_OF_MEMORY, "cudaMallocAsync(%zu) for the decoded keys: %s", need,
-                    cudaGetErrorString(e));
-      }
+      st = scratch_alloc(&kraw, need, cs, "the decoded MXFP4 keys");
+      if (st != SI_OK) return st;
       base = kraw;
     }
     void* kdec = reinterpret_cast<void*>((reinterpret_cast<uintptr_t>(base) + 255) & ~static_cast<uintptr_t>(255));
@@ -183,7 +251,8 @@ si_status stream_topk_rows(const void* q, const void* kc, const float* w, int B,
   }
   if (st == SI_OK) st = launch_stream_topk(q, kc, w, B, S, T, H_I, D, m, k, out_idx, out_score, cs, cfg);
   // the kernel leaves each row's k results in pool order: sort them now
-  if (st == SI_OK && !cfg.unsorted && out_score)
+  // (rows that went through the split-key merge are sorted already)
+  if (st == SI_OK && !cfg.unsorted && out_score && !sorted_by_merge)
     st = launch_row_sort(out_idx, out_score, static_cast<long long>(B) * S, k, cs);
   if (kraw) {
     const cudaError_t e = cudaFreeAsync(kraw, cs);
@@ -192,7 +261,9 @@ si_status stream_topk_rows(const void* q, const void* kc, const float* w, int B,
   return st;
 }
 
-}  // namespace
+}  // namespace si
+
+using namespace si;
 
 extern "C" {
 
@@ -229,7 +300,7 @@ si_status si_indexer_topk(const void* q, const void* kc, const float* w, int B, 
 // bounded waits run out and it exits with SI_ERR_TIMEOUT recorded.
 si_status si_test_stream_timeout(const void* q, const void* kc, const float* w, int B, int S, int T,
                                  int m, int k, int32_t* out_idx, void* stream,
-                                 unsigned long long wait_limit_ns) {
+                                 unsigned long long wait_limit_ns, int32_t* device_status) {
   si_status st = check_common(q, kc, w, B, S, T, 64, 128, m, k, out_idx, nullptr);
   if (st != SI_OK) return st;
   StreamConfig cfg;
@@ -241,6 +312,11 @@ si_status si_test_stream_timeout(const void* q, const void* kc, const float* w, 
   cfg.wait_limit_ns = wait_limit_ns;
   cfg.test_withhold = 1;
   cfg.unsorted = false;
+  si_options o;
+  std::memset(&o, 0, sizeof o);
+  o.device_status = device_status;
+  st = error_word(&o, &cfg.err);
+  if (st != SI_OK) return st;
   return launch_stream_topk(q, kc, w, B, S, T, 64, 128, m, k, out_idx, nullptr,
                             static_cast<cudaStream_t>(stream), cfg);
 }
@@ -261,10 +337,16 @@ si_status si_indexer_materialize(const void* q, const void* kc, const float* w, 
 size_t si_indexer_workspace_size(int B, int S, int T, int H_I, int D, int m, int k, int materialize,
                                  const si_options* opt) {
   (void)m;
-  (void)k;
-  if (B < 1 || S < 1 || T < 1 || H_I < 1 || D < 1) return 0;
+  if (B < 1 || S < 1 || T < 1 || H_I < 1 || D < 1 || k < 1) return 0;
   if (materialize) return materialize_workspace_bytes(B, S, T, H_I);
-  return opt && opt->dtype == SI_DTYPE_MXFP4_KEYS ? mxfp4_key_bytes(B, T, D) : 0;
+  int dev = 0, n_sm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    n_sm = 1024;  // no device to ask: a bound for any GPU
+  }
+  const size_t mxb = opt && opt->dtype == SI_DTYPE_MXFP4_KEYS ? mxfp4_key_bytes(B, T, D) : 0;
+  return mxb + stream_split_bytes_bound(B, S, k, opt ? opt->query_chunk : 0, n_sm);
 }
 
 size_t si_two_stage_workspace_size(int B, int S, int T, int block, int n_keep, int query_chunk) {
@@ -287,9 +369,36 @@ si_status si_indexer_topk_two_stage(const void* q, const void* kc, const float* 
   if (static_cast<long long>(m) * block > 0x7FFFFFFFll || static_cast<long long>(B) * S * H_I > 0x7FFFFFFFll)
     return fail(SI_ERR_UNSUPPORTED, "m*block and B*S*H_I must fit in 31 bits");
   const int chunk = opt && opt->query_chunk > 0 ? opt->query_chunk : 16384;
+  int* err = nullptr;
+  st = error_word(opt, &err);
+  if (st != SI_OK) return st;
   return launch_two_stage(q, kc, w, B, S, T, m, k, block, n_keep, chunk, out_idx, out_score,
                           opt ? opt->workspace : nullptr, opt ? opt->workspace_bytes : 0, kDefaultWaitLimitNs,
-                          static_cast<cudaStream_t>(stream));
+                          err, static_cast<cudaStream_t>(stream));
+}
+
+si_status si_sparse_attention(const void* q, const void* kv, const int32_t* idx, int B, int S, int T, int H,
+                              int Dk, int Dv, int k, float scale, void* out, float* lse, void* stream,
+                              const si_options* opt) {
+  if (!q || !kv || !idx || !out || !lse)
+    return fail(SI_ERR_INVALID_ARGUMENT, "q, kv, idx, out and lse must be non-null device pointers");
+  if (B < 1 || S < 1 || T < 1 || H < 1 || Dk < 1 || Dv < 1 || k < 1)
+    return fail(SI_ERR_INVALID_ARGUMENT, "B, S, T, H, Dk, Dv, k must be >= 1");
+  if (!aligned(q, 16) || !aligned(kv, 16) || !aligned(idx, 16) || !aligned(out, 16) || !aligned(lse, 4))
+    return fail(SI_ERR_INVALID_ARGUMENT, "q, kv, idx, out must be 16-byte aligned; lse 4-byte aligned");
+  if (!(scale >= 0.f) || scale != scale)
+    return fail(SI_ERR_INVALID_ARGUMENT, "scale must be >= 0 (0 = 1/sqrt(Dk))");
+  if (H != 64 || Dk != 576 || Dv != 512)
+    return fail(SI_ERR_UNSUPPORTED, "sparse attention implements H=64, Dk=576, Dv=512 (got %d, %d, %d)", H, Dk, Dv);
+  if (k % 128 != 0 || k > 512) return fail(SI_ERR_UNSUPPORTED, "k must be 128, 256, 384 or 512 (got %d)", k);
+  if (static_cast<long long>(B) * S * H > 0x7FFFFFFFll || static_cast<long long>(B) * T > 0x7FFFFFFFll)
+    return fail(SI_ERR_UNSUPPORTED, "B*S*H and B*T must fit in 31 bits");
+  int* err = nullptr;
+  si_status st = error_word(opt, &err);
+  if (st != SI_OK) return st;
+  const float sc = scale > 0.f ? scale : 1.0f / sqrtf(static_cast<float>(Dk));
+  return launch_sparse_attention(q, kv, idx, B, S, T, k, sc, out, lse, err, kDefaultWaitLimitNs,
+                                 static_cast<cudaStream_t>(stream));
 }
 
 si_status si_mxfp4_to_bf16(const void* codes, const void* scales, int64_t rows, int D, void* out,
@@ -334,6 +443,8 @@ const char* si_status_string(si_status s) {
 }
 
 const char* si_last_error(void) { return g_last_error; }
+
+void si_test_fail_allocations(int n) { g_fail_allocs.store(n > 0 ? n : 0); }
 
 int si_version(void) { return 300; }
 

@@ -1,0 +1,446 @@
+// Sparse attention over the indexer's selected compressed latents (the
+// consumer of the top-k).
+//
+// StreamIndex (abstract): the sparse attention kernel reads only the entries
+// the indexer selected.  Reading of the pages (DeepSeek-V3.2 lineage that the
+// V4.1 page gives): every one of the H = 64 heads of query t attends over the
+// k selected compressed latents of its sequence; a latent is the key (all
+// Dk = 576 values: 512 latent + 64 rope) and the value (its first Dv = 512);
+// the softmax runs over the selection only with scale 1/sqrt(Dk) (or the
+// caller's); index -1 is padding; a row with nothing selected gives O = 0 and
+// lse = -inf.
+//
+// One CTA per SM, persistent over queries.  Per query:
+//   QK   S^T[e, h] = sum_d kv[sel[e], d] * q[h, d]: tcgen05 kind::f16, A = 128
+//        gathered latent rows (M = entries) x 64 dims per stage, SW128
+//        K-major; B = q[t] (N = 64 heads, K = 576) TMA-loaded once; fp32 into
+//        TMEM columns [64 j, 64 j + 64) for entry tile j.
+//   soft max and sum per head over the k entries (4 softmax warps, lane =
+//        entry, 32 heads at a time), P = exp(scale (s - max)) rounded to bf16
+//        and written as P^T (N = heads, K = entries, SW128 K-major), the sums
+//        of the rounded P kept for the normalisation, lse = scale max + ln sum.
+//   PV   O^T[dv, h] = sum_e V[e, dv] P^T[h, e]: A = gathered value tiles read
+//        MN-major (M = dv, contiguous in each latent row; 128 dv x 64 entries
+//        per stage), B = P^T; fp32 into TMEM columns [256 + 64 v, ...) for dv
+//        tile v.
+//   out  O[t, h, dv] = O^T * (1 / sum_h), bf16; lse[t, h] fp32.
+// Warps: 0 q loads (TMA), 1 MMA issue, 2-3 gather producers (16-byte
+// cp.async into the swizzled stages), 4-7 softmax and epilogue.  Every wait
+// is bounded; on expiry the kernel records SI_ERR_TIMEOUT, drains its copies
+// and MMAs and exits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+
+#include "si_internal.h"
+#include "si_ptx.cuh"
+
+namespace si {
+namespace {
+
+constexpr int A_H = 64, A_DK = 576, A_DV = 512, A_KMAX = 512;
+constexpr int A_KB = A_DK / 64;             // 9 K-blocks of 64 dims
+constexpr int A_THREADS = 256;
+constexpr int A_NS = 4;                     // gather stages of 16 KB
+constexpr int A_STAGE = 16384;
+constexpr int A_Q_BYTES = A_H * A_DK * 2;   // 72 KB: 9 blocks of [64 rows x 128 B]
+constexpr int A_P_BYTES = A_H * A_KMAX * 2; // 64 KB: up to 8 blocks of [64 heads x 128 B]
+
+enum { AERR_Q_FREE = 21, AERR_Q_FULL = 22, AERR_STAGE_FREE = 23, AERR_STAGE_FULL = 24, AERR_S_FULL = 25,
+       AERR_P_FULL = 26, AERR_O_FULL = 27, AERR_O_FREE = 28, AERR_DRAIN = 29 };
+
+struct AttnParams {
+  const uint8_t* kv;      // [B, T, 576] bf16 bytes
+  const int32_t* idx;     // [B, S, k]
+  __nv_bfloat16* out;     // [B, S, 64, 512]
+  float* lse;             // [B, S, 64]
+  int* err;
+  int B, S, T, k;
+  float scale;
+  uint64_t wait_limit_ns;
+};
+
+struct ACtrl {
+  uint64_t full[A_NS], empty[A_NS];
+  uint64_t q_full, q_empty, s_full, p_full, o_full, o_empty, done;
+  uint32_t tmem_slot;
+  int abort;
+  float red[4][A_H];      // per-quadrant partial max / sum
+  float head_max[A_H], head_inv[A_H];  // per head: max logit, 1 / sum of the rounded weights
+};
+
+__device__ __forceinline__ void cp16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+// Shared-memory descriptor of an MN-major operand with the 128-byte swizzle:
+// atoms of 8 K-rows x 128 bytes (64 bf16 along M/N); `lbo` = bytes between
+// atoms along M/N, `sbo` = bytes between 8-row groups along K (the canonical
+// MN-major layout of the tcgen05 matrix descriptor, version 1).
+__device__ __forceinline__ uint64_t sdesc_mnmajor_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  d |= static_cast<uint64_t>(2u) << 61;
+  return d;
+}
+
+__device__ __forceinline__ void attn_error(const AttnParams& p, volatile int* abort, int where) {
+  atomicCAS(p.err, 0, static_cast<int>(SI_ERR_TIMEOUT));
+  atomicCAS(p.err + 1, 0, where);
+  *abort = 1;
+}
+
+__global__ void __launch_bounds__(A_THREADS, 1)
+    sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const AttnParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* q_s = smem;
+  uint8_t* st_s = smem + A_Q_BYTES;
+  uint8_t* p_s = st_s + A_NS * A_STAGE;
+  ACtrl* C = reinterpret_cast<ACtrl*>(p_s + A_P_BYTES);
+  volatile int* abort = &C->abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_et = p.k / 128;            // entry tiles of the QK product
+  const int n_kc = p.k / 64;             // 64-entry chunks of the PV product
+  const int qk_stages = n_et * A_KB, pv_stages = 4 * n_kc;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < A_NS; ++s) {
+      mbar_init(&C->full[s], 64);
+      mbar_init(&C->empty[s], 1);
+    }
+    mbar_init(&C->q_full, 1);
+    mbar_init(&C->q_empty, 1);
+    mbar_init(&C->s_full, 1);
+    mbar_init(&C->p_full, 128);
+    mbar_init(&C->o_full, 1);
+    mbar_init(&C->o_empty, 128);
+    mbar_init(&C->done, 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) prefetch_tmap(&tm_q);
+  if (warp == 1) tmem_alloc(&C->tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = C->tmem_slot;
+  const int nq = p.B * p.S;               // queries, sequence-major
+  const int q0 = blockIdx.x, qstep = gridDim.x;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ q rows (TMA)
+      uint32_t n = 0;
+      for (int t = q0; t < nq; t += qstep, ++n) {
+        if (!mbar_wait_bounded(&C->q_empty, (n & 1u) ^ 1u, abort, p.wait_limit_ns)) {
+          attn_error(p, abort, AERR_Q_FREE);
+          break;
+        }
+        mbar_arrive_expect_tx(&C->q_full, A_Q_BYTES);
+        for (int kb = 0; kb < A_KB; ++kb) tma_load_2d(q_s + kb * 8192, &tm_q, &C->q_full, kb * 64, t * A_H);
+      }
+      if (n && !mbar_wait_timed(&C->q_full, (n - 1) & 1u, p.wait_limit_ns)) attn_error(p, abort, AERR_DRAIN);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
+      constexpr uint32_t IDESC_QK = idesc_f32acc(1, 1, 128, A_H);
+      constexpr uint32_t IDESC_PV = idesc_f32acc(1, 1, 128, A_H) | (1u << 15);  // A (V^T) MN-major
+      const uint32_t qa = smem_u32(q_s), sa = smem_u32(st_s), pa = smem_u32(p_s);
+      uint32_t stage = 0, phase = 0, n = 0;
+      bool stop = false;
+      for (int t = q0; t < nq && !stop; t += qstep, ++n) {
+        const uint32_t par = n & 1u;
+        if (!mbar_wait_bounded(&C->q_full, par, abort, p.wait_limit_ns)) {
+          attn_error(p, abort, AERR_Q_FULL);
+          break;
+        }
+        tc_fence_after();
+        for (int jt = 0; jt < n_et && !stop; ++jt)
+          for (int kb = 0; kb < A_KB; ++kb) {
+            if (!mbar_wait_bounded(&C->full[stage], phase, abort, p.wait_limit_ns)) {
+              attn_error(p, abort, AERR_STAGE_FULL);
+              stop = true;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a0 = sa + stage * A_STAGE;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16(tmem + jt * A_H, sdesc_kmajor_sw128(a0 + kk * 32), sdesc_kmajor_sw128(qa + kb * 8192 + kk * 32),
+                       IDESC_QK, (kb | kk) != 0);
+            mma_commit(&C->empty[stage]);
+            if (++stage == A_NS) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+        if (stop) break;
+        mma_commit(&C->s_full);
+        mma_commit(&C->q_empty);
+        if (!mbar_wait_bounded(&C->p_full, par, abort, p.wait_limit_ns)) {
+          attn_error(p, abort, AERR_P_FULL);
+          break;
+        }
+        if (!mbar_wait_bounded(&C->o_empty, par ^ 1u, abort, p.wait_limit_ns)) {
+          attn_error(p, abort, AERR_O_FREE);
+          break;
+        }
+        tc_fence_after();
+        for (int vt = 0; vt < 4 && !stop; ++vt)
+          for (int c = 0; c < n_kc; ++c) {
+            if (!mbar_wait_bounded(&C->full[stage], phase, abort, p.wait_limit_ns)) {
+              attn_error(p, abort, AERR_STAGE_FULL);
+              stop = true;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a0 = sa + stage * A_STAGE;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)  // 16 entries a step: two 8-entry atom rows
+              mma_bf16(tmem + 256 + vt * A_H, sdesc_mnmajor_sw128(a0 + kk * 2048, 8192, 1024),
+                       sdesc_kmajor_sw128(pa + c * 8192 + kk * 32), IDESC_PV, (c | kk) != 0);
+            mma_commit(&C->empty[stage]);
+            if (++stage == A_NS) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+        if (!stop) mma_commit(&C->o_full);
+      }
+      // every MMA issued above has completed before TMEM is released
+      mma_commit(&C->done);
+      if (!mbar_wait_timed(&C->done, 0, p.wait_limit_ns)) attn_error(p, abort, AERR_DRAIN);
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ gather producers
+    const int pt = threadIdx.x - 64;
+    uint32_t stage = 0, phase = 0;
+    int pend[3], np = 0;
+    bool stop = false;
+    for (int t = q0; t < nq && !stop; t += qstep) {
+      const int b = t / p.S;
+      const int32_t* sel = p.idx + static_cast<size_t>(t) * p.k;
+      const uint8_t* kvb = p.kv + static_cast<size_t>(b) * p.T * (A_DK * 2);
+      for (int j = 0; j < qk_stages + pv_stages; ++j) {
+        const bool got = mbar_wait_bounded(&C->empty[stage], phase ^ 1u, abort, p.wait_limit_ns);
+        if (!__all_sync(0xFFFFFFFFu, got)) {
+          if (lane == 0) attn_error(p, abort, AERR_STAGE_FREE);
+          stop = true;
+          break;
+        }
+        const uint32_t base = smem_u32(st_s + stage * A_STAGE);
+#pragma unroll 4
+        for (int i = 0; i < 16; ++i) {
+          const int id = pt + 64 * i, ch = id & 7;
+          int row, e, col_bytes, a = 0;
+          if (j < qk_stages) {             // entry tile j / 9, K-block j % 9: 128 rows x 128 B
+            row = id >> 3;
+            e = (j / A_KB) * 128 + row;
+            col_bytes = (j % A_KB) * 128;
+          } else {                         // dv tile, 64-entry chunk: 2 atoms (64 dv each) x 64 rows x 128 B
+            const int jj = j - qk_stages;
+            a = id >> 9;
+            row = (id >> 3) & 63;
+            e = (jj % n_kc) * 64 + row;
+            col_bytes = ((jj / n_kc) * 128 + a * 64) * 2;
+          }
+          int key = sel[e];
+          key = key >= 0 && key < p.T ? key : 0;  // padding reads row 0; its weight is 0
+          cp16(base + a * 8192 + row * 128 + ((ch ^ (row & 7)) << 4),
+               kvb + static_cast<size_t>(key) * (A_DK * 2) + col_bytes + ch * 16);
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        pend[np++] = static_cast<int>(stage);
+        if (np == 3) {
+          asm volatile("cp.async.wait_group 2;" ::: "memory");
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          mbar_arrive(&C->full[pend[0]]);
+          pend[0] = pend[1];
+          pend[1] = pend[2];
+          np = 2;
+        }
+        if (++stage == A_NS) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    for (int e = 0; e < np; ++e) mbar_arrive(&C->full[pend[e]]);
+  } else {
+    // ------------------------------------------------------------ softmax + epilogue
+    // The four warps meet at named barriers, so none may leave the loop early:
+    // after a failed wait a warp keeps going through every barrier with ok =
+    // false and touches neither TMEM nor the outputs.
+    const int quad = warp - 4;
+    const float ninf = -__int_as_float(0x7f800000);
+    uint32_t n = 0;
+    bool ok = true;
+    for (int t = q0; t < nq; t += qstep, ++n) {
+      const uint32_t par = n & 1u;
+      bool valid[4];
+#pragma unroll
+      for (int jt = 0; jt < 4; ++jt) {
+        const int e = jt * 128 + quad * 32 + lane;
+        valid[jt] = jt < n_et && p.idx[static_cast<size_t>(t) * p.k + e] >= 0 &&
+                    p.idx[static_cast<size_t>(t) * p.k + e] < p.T;
+      }
+      const bool got = ok && mbar_wait_bounded(&C->s_full, par, abort, p.wait_limit_ns);
+      if (ok && !__all_sync(0xFFFFFFFFu, got)) {
+        if (lane == 0) attn_error(p, abort, AERR_S_FULL);
+        ok = false;
+      }
+      tc_fence_after();
+      // two passes of 32 heads keep the live arrays at 3 x 32 registers
+      for (int hh = 0; hh < 2; ++hh) {
+        float m[32], sum[32];
+        uint32_t x[32];
+#pragma unroll
+        for (int h = 0; h < 32; ++h) m[h] = ninf;
+#pragma unroll
+        for (int jt = 0; jt < 4; ++jt) {
+          if (jt >= n_et || !ok) break;
+          tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + jt * A_H + hh * 32, x);
+          tmem_ld_wait();
+          if (valid[jt]) {
+#pragma unroll
+            for (int h = 0; h < 32; ++h) m[h] = fmaxf(m[h], __uint_as_float(x[h]));
+          }
+        }
+#pragma unroll
+        for (int h = 0; h < 32; ++h)
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) m[h] = fmaxf(m[h], __shfl_xor_sync(0xFFFFFFFFu, m[h], o));
+        {
+          float mine = 0.f;  // m[lane] without a dynamic register index
+#pragma unroll
+          for (int h = 0; h < 32; ++h) mine = h == lane ? m[h] : mine;
+          C->red[quad][hh * 32 + lane] = mine;
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+#pragma unroll
+        for (int h = 0; h < 32; ++h) {
+          const int hg = hh * 32 + h;
+          m[h] = fmaxf(fmaxf(C->red[0][hg], C->red[1][hg]), fmaxf(C->red[2][hg], C->red[3][hg]));
+        }
+        if (quad == 0) {
+          float mine = 0.f;
+#pragma unroll
+          for (int h = 0; h < 32; ++h) mine = h == lane ? m[h] : mine;
+          C->head_max[hh * 32 + lane] = mine;
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");  // red is reused for the sums
+#pragma unroll
+        for (int h = 0; h < 32; ++h) sum[h] = 0.f;
+#pragma unroll
+        for (int jt = 0; jt < 4; ++jt) {
+          if (jt >= n_et || !ok) break;
+          tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + jt * A_H + hh * 32, x);
+          tmem_ld_wait();
+          const int e = jt * 128 + quad * 32 + lane, kb = e >> 6, col = e & 63;
+#pragma unroll
+          for (int h = 0; h < 32; ++h) {
+            const int hg = hh * 32 + h;
+            const float pr = valid[jt] ? __expf(p.scale * (__uint_as_float(x[h]) - m[h])) : 0.f;
+            const __nv_bfloat16 pb = __float2bfloat16_rn(pr);
+            sum[h] += __bfloat162float(pb);
+            // P^T K-major: block kb = [64 heads][64 entries], row hg, swizzled 16-byte chunk
+            const int off = kb * 8192 + hg * 128 + ((((col * 2) >> 4) ^ (hg & 7)) << 4) + ((col * 2) & 15);
+            *reinterpret_cast<__nv_bfloat16*>(p_s + off) = pb;
+          }
+        }
+#pragma unroll
+        for (int h = 0; h < 32; ++h)
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) sum[h] += __shfl_xor_sync(0xFFFFFFFFu, sum[h], o);
+        {
+          float mine = 0.f;
+#pragma unroll
+          for (int h = 0; h < 32; ++h) mine = h == lane ? sum[h] : mine;
+          C->red[quad][hh * 32 + lane] = mine;
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (quad == 0) {
+          const int hg = hh * 32 + lane;
+          const float s = C->red[0][hg] + C->red[1][hg] + C->red[2][hg] + C->red[3][hg];
+          C->head_inv[hg] = s > 0.f ? 1.0f / s : 0.f;
+          if (ok) p.lse[static_cast<size_t>(t) * A_H + hg] = s > 0.f ? p.scale * C->head_max[hg] + __logf(s) : ninf;
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // P is read by the MMA (async proxy)
+      tc_fence_before();
+      mbar_arrive(&C->p_full);
+      // epilogue: lane = dv, 64 heads a load
+      const bool gotO = ok && mbar_wait_bounded(&C->o_full, par, abort, p.wait_limit_ns);
+      if (ok && !__all_sync(0xFFFFFFFFu, gotO)) {
+        if (lane == 0) attn_error(p, abort, AERR_O_FULL);
+        ok = false;
+      }
+      tc_fence_after();
+      uint32_t x[64];
+      for (int vt = 0; vt < 4 && ok; ++vt) {
+        tmem_ld32_x64(tmem + (static_cast<uint32_t>(quad * 32) << 16) + 256 + vt * A_H, x);
+        tmem_ld_wait();
+        const int dv = vt * 128 + quad * 32 + lane;
+#pragma unroll
+        for (int h = 0; h < A_H; ++h)
+          p.out[(static_cast<size_t>(t) * A_H + h) * A_DV + dv] =
+              __float2bfloat16_rn(__uint_as_float(x[h]) * C->head_inv[h]);
+      }
+      tc_fence_before();
+      mbar_arrive(&C->o_empty);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace
+
+si_status launch_sparse_attention(const void* q, const void* kv, const int32_t* idx, int B, int S, int T, int k,
+                                  float scale, void* out, float* lse, int* err, uint64_t wait_limit_ns,
+                                  cudaStream_t stream) {
+  CUtensorMap tm_q;
+  si_status st = encode_tmap_2d(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, A_DK,
+                                static_cast<uint64_t>(B) * S * A_H, A_DK * 2, 64, A_H);
+  if (st != SI_OK) return st;
+  int dev = 0, n_sm = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "device query");
+  const size_t smem = 1024 + A_Q_BYTES + A_NS * A_STAGE + A_P_BYTES + sizeof(ACtrl);
+  e = cudaFuncSetAttribute(sparse_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(sparse_attn_kernel)");
+  AttnParams p;
+  p.kv = static_cast<const uint8_t*>(kv);
+  p.idx = idx;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.err = err;
+  p.B = B;
+  p.S = S;
+  p.T = T;
+  p.k = k;
+  p.scale = scale;
+  p.wait_limit_ns = wait_limit_ns;
+  const long long nq = static_cast<long long>(B) * S;
+  const int grid = static_cast<int>(std::min<long long>(nq, n_sm));
+  sparse_attn_kernel<<<grid, A_THREADS, smem, stream>>>(tm_q, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "sparse_attn_kernel launch");
+  return SI_OK;
+}
+
+}  // namespace si

@@ -171,11 +171,8 @@ si_status launch_materialize(const void* q, const void* kc, const float* w, int 
       return fail(SI_ERR_OUT_OF_MEMORY,
                   "materialize needs %zu bytes for the [B,S,H_I,T] logits and [B,S,T] scores; %zu free",
                   need, free_b);
-    e = cudaMallocAsync(&ws, need, stream);
-    if (e != cudaSuccess) {
-      cudaGetLastError();
-      return fail(SI_ERR_OUT_OF_MEMORY, "cudaMallocAsync(%zu): %s", need, cudaGetErrorString(e));
-    }
+    const si_status sa = scratch_alloc(&ws, need, stream, "the materialized logits and scores");
+    if (sa != SI_OK) return sa;
     owned = true;
   }
   float* L = static_cast<float*>(ws);

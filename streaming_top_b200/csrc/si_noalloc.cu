@@ -10,16 +10,20 @@
 // materialize kernels with their [B,S,H_I,T] logits and [B,S,T] scores placed
 // in a fixed device array of this file instead of memory allocated per call.
 //
-// The array is SI_NOALLOC_SCRATCH_BYTES (64 MiB); every GPU that loads the
-// library holds it until the process exits.  Problems whose scratch need,
-// 4*B*S*T*(H_I+1) + 256 bytes, exceeds it are rejected.  All calls share the
-// array and it keeps the last call's contents; the kernels overwrite every
-// word they read before reading it, so nothing needs clearing.  Each device
-// has its own copy; two calls on one device whose work overlaps on the GPU
-// (on different streams, say) race on it, so serialise them.
+// The array is SI_NOALLOC_SCRATCH_BYTES (64 MiB) on every GPU where the
+// library's module is loaded, held until the process exits.  Under CUDA's
+// lazy module loading (the default) that happens at the first call of this
+// entry point on the device, which therefore itself needs the 64 MiB free:
+// a caller whose pool is about to take nearly all memory makes one call
+// first (any small problem) to reserve it.  If the reservation fails the
+// call returns SI_ERR_OUT_OF_MEMORY.  Problems whose scratch need,
+// 4*B*S*T*(H_I+1) + 256 bytes, exceeds the array are rejected.  All calls
+// share the array and it keeps the last call's contents; the kernels
+// overwrite every word they read before reading it, so nothing needs
+// clearing.  Each device has its own copy; two calls on one device whose
+// work overlaps on the GPU (on different streams, say) race on it, so
+// serialise them.
 #include <cuda_runtime.h>
-
-#include <mutex>
 
 #include "si_internal.h"
 
@@ -28,26 +32,23 @@ namespace {
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[SI_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void* g_scratch[kMaxDevices] = {};
-
-// Device address of the scratch array on the current device.  Host code only
-// sees a host-side stand-in for the array's name, so the address is asked
-// for once per device, with that device current, and cached.
+// Device address of the scratch array in the current context.  Host code
+// only sees a host-side stand-in for the array's name, so the address is
+// asked for on every call, with the caller's device current: no cached
+// pointer can outlive a device reset or belong to another context.  The
+// first lookup on a device loads the module and so reserves the array.
 si_status scratch_address(void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  if (dev < 0 || dev >= kMaxDevices) return fail(SI_ERR_UNSUPPORTED, "device index %d", dev);
-  std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_scratch[dev]) {
-    void* ptr = nullptr;
-    e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
-    g_scratch[dev] = ptr;
+  void* ptr = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+  if (e == cudaErrorMemoryAllocation) {
+    cudaGetLastError();
+    return fail(SI_ERR_OUT_OF_MEMORY,
+                "reserving the %zu-byte no-alloc scratch array on this device failed (%s); make the "
+                "first call before other allocations fill the device",
+                static_cast<size_t>(SI_NOALLOC_SCRATCH_BYTES), cudaGetErrorString(e));
   }
-  *out = g_scratch[dev];
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
+  *out = ptr;
   return SI_OK;
 }
 

@@ -112,19 +112,36 @@ struct Params {
   int sort_rows;          // finalize sorts each row itself (no scores to sort by later)
 };
 
-struct Unit {
-  int b, t0, n_keys, n_kt;
+// A work item: one unit (4 consecutive queries of one sequence) and, when
+// the unit's keys are split over CTAs, one contiguous range of its key
+// tiles [kt0, kt1).
+struct SplitParams {
+  int n_split;            // key partitions per unit, each on its own CTA (1: none)
+  int32_t* part_idx;      // n_split > 1: per-partition top-k [B][part_rows][n_split][k]
+  float* part_score;
+  int part_rows;          // rows per sequence in the partials (the launch's query tiles x 4)
 };
 
-__device__ __forceinline__ Unit decode_unit(int u, const Params& p) {
+struct Unit {
+  int b, t0, n_keys, kt0, kt1, sp;
+};
+
+// SPLIT: the launch splits units' keys over CTAs (n_split partitions); the
+// other instantiation keeps whole units (n_split == 1) and pays nothing for it.
+template <bool SPLIT>
+__device__ __forceinline__ Unit decode_unit(int w, const Params& p, const SplitParams& x) {
   Unit r;
+  const int u = SPLIT ? w / x.n_split : w;
+  r.sp = SPLIT ? w - u * x.n_split : 0;
   r.b = u % p.B;
   const int qt = p.qt_end - 1 - u / p.B;
   r.t0 = qt * QT;
   const int t_last = min(r.t0 + QT, p.S) - 1;
   const int n = (p.row0 + t_last + 1) / p.m;
   r.n_keys = n < p.T ? n : p.T;
-  r.n_kt = (r.n_keys + KT - 1) / KT;
+  const int n_kt = (r.n_keys + KT - 1) / KT;
+  r.kt0 = SPLIT ? static_cast<int>(static_cast<long long>(r.sp) * n_kt / x.n_split) : 0;
+  r.kt1 = SPLIT ? static_cast<int>(static_cast<long long>(r.sp + 1) * n_kt / x.n_split) : n_kt;
   return r;
 }
 
@@ -240,10 +257,10 @@ struct Ctrl {
 };
 static_assert(sizeof(Ctrl) <= CTRL_BYTES, "control block");
 
-template <int OPB>
+template <int OPB, bool SPLIT>
 __global__ void __launch_bounds__(THREADS, 1)
     stream_topk_kernel(const __grid_constant__ CUtensorMap tm_q,
-                       const __grid_constant__ CUtensorMap tm_kc, const Params p) {
+                       const __grid_constant__ CUtensorMap tm_kc, const Params p, const SplitParams x) {
   using L = Layout<OPB>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -290,7 +307,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = C->tmem_slot;
 
-  const int n_units = p.B * (p.qt_end - p.qt_begin);
+  const int n_units = p.B * (p.qt_end - p.qt_begin) * (SPLIT ? x.n_split : 1);  // work items
   const int q_bytes = L::Q_BYTES, kc_bytes = L::KC_BYTES;
 
   if (warp < 4) {
@@ -304,8 +321,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int i = 0;; ++i) {
         const int u = unit_of(i, n_units);
         if (u < 0 || *abort) break;
-        const Unit U = decode_unit(u, p);
-        if (U.n_kt == 0) continue;
+        const Unit U = decode_unit<SPLIT>(u, p, x);
+        if (U.kt1 == U.kt0) continue;
         if (!mbar_wait_bounded(&C->q_empty, qph ^ 1u, abort, p.wait_limit_ns)) {
           record_error(p, abort, ERR_WAIT_QFREE);
           break;
@@ -317,7 +334,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         ++q_issued;
         qph ^= 1u;
         bool stop = false;
-        for (int j = 0; j < U.n_kt; ++j) {
+        for (int j = U.kt0; j < U.kt1; ++j) {
           if (!mbar_wait_bounded(&C->empty[stage], phase ^ 1u, abort, p.wait_limit_ns)) {
             record_error(p, abort, ERR_WAIT_KFREE);
             stop = true;
@@ -357,8 +374,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int i = 0;; ++i) {
         const int u = unit_of(i, n_units);
         if (u < 0 || *abort) break;
-        const Unit U = decode_unit(u, p);
-        if (U.n_kt == 0) continue;
+        const Unit U = decode_unit<SPLIT>(u, p, x);
+        if (U.kt1 == U.kt0) continue;
         if (!mbar_wait_bounded(&C->q_full, qph, abort, p.wait_limit_ns)) {
           record_error(p, abort, ERR_WAIT_Q);
           break;
@@ -366,7 +383,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         qph ^= 1u;
         tc_fence_after();
         bool stop = false;
-        for (int j = 0; j < U.n_kt; ++j) {
+        for (int j = U.kt0; j < U.kt1; ++j) {
           if (!mbar_wait_bounded(&C->t_empty[acc], accph ^ 1u, abort, p.wait_limit_ns)) {
             record_error(p, abort, ERR_WAIT_TMEM_EMPTY);
             stop = true;
@@ -392,7 +409,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
           mma_commit(&C->empty[stage]);
           mma_commit(&C->t_full[acc]);
-          if (j == U.n_kt - 1) mma_commit(&C->q_empty);
+          if (j == U.kt1 - 1) mma_commit(&C->q_empty);
           if (++stage == static_cast<uint32_t>(p.n_stages)) {
             stage = 0;
             phase ^= 1u;
@@ -423,7 +440,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int i = 0;; ++i) {
       const int u = unit_of(i, n_units);
       if (u < 0) break;
-      const Unit U = decode_unit(u, p);
+      const Unit U = decode_unit<SPLIT>(u, p, x);
       if (lane == 0) {
         st->cnt = 0;
         st->thr = 0;
@@ -434,7 +451,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       __syncwarp();
       const int t = U.t0 + q;
       int in_part = 0;
-      for (int j = 0; j < U.n_kt; ++j, ++tix) {
+      for (int j = U.kt0; j < U.kt1; ++j, ++tix) {
         const uint32_t slot = tix & (RING - 1), par = (tix / RING) & 1u;
         if (ok && !*abort && !mbar_wait_bounded(&C->ring_full[slot], par, abort, p.wait_limit_ns)) {
           record_error(p, abort, ERR_WAIT_RING_FULL);
@@ -452,7 +469,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&C->ring_free[slot]);  // the slot has been read
-        const bool last = j == U.n_kt - 1;
+        const bool last = j == U.kt1 - 1;
         if (++in_part == tpp || last) {
           in_part = 0;
           // at the unit's end only a histogram that does not exist yet is worth
@@ -468,9 +485,16 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (t < p.S) {
         if (!ok && lane == 0) st->cnt = 0;  // after an abort: contents unspecified
         __syncwarp();
-        const size_t ob = (static_cast<size_t>(U.b) * p.S + t) * static_cast<size_t>(k);
-        topk::finalize(st, pool, qh, k, p.out_idx + ob, p.out_score ? p.out_score + ob : nullptr,
-                       p.sort_rows != 0, lane);
+        if (SPLIT) {
+          // this key partition's exact top-k, for the merge kernel
+          const size_t pr = static_cast<size_t>(U.b) * x.part_rows + (t - p.qt_begin * QT);
+          const size_t ob = (pr * x.n_split + U.sp) * static_cast<size_t>(k);
+          topk::finalize(st, pool, qh, k, x.part_idx + ob, x.part_score + ob, false, lane);
+        } else {
+          const size_t ob = (static_cast<size_t>(U.b) * p.S + t) * static_cast<size_t>(k);
+          topk::finalize(st, pool, qh, k, p.out_idx + ob, p.out_score ? p.out_score + ob : nullptr,
+                         p.sort_rows != 0, lane);
+        }
       }
     }
   } else {
@@ -486,8 +510,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int i = 0;; ++i) {
       const int u = unit_of(i, n_units);
       if (u < 0) break;
-      const Unit U = decode_unit(u, p);
-      if (U.n_kt == 0) continue;
+      const Unit U = decode_unit<SPLIT>(u, p, x);
+      if (U.kt1 == U.kt0) continue;
       // the two queries' head weights (times the q scales for fp8) into this
       // warp's table, 0 for queries past the end of the sequence; the first
       // query's then go to registers
@@ -525,8 +549,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       // fp8: the key scales of the next tile are fetched one tile ahead
       const float* ks_row = OPB == 1 ? p.kc_scale + static_cast<size_t>(U.b) * p.T : nullptr;
       float ksc_next = 1.f;
-      if (OPB == 1 && key_off < p.T) ksc_next = ks_row[key_off];
-      for (int j = 0; j < U.n_kt; ++j, ++tix) {
+      if (OPB == 1 && U.kt0 * KT + key_off < p.T) ksc_next = ks_row[U.kt0 * KT + key_off];
+      for (int j = U.kt0; j < U.kt1; ++j, ++tix) {
         ok = ok && !*abort;
         if (ok && !mbar_wait_bounded(&C->t_full[acc], accph, abort, p.wait_limit_ns)) {
           record_error(p, abort, ERR_WAIT_TMEM_FULL);
@@ -538,7 +562,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           tc_fence_after();
           const uint32_t ta = tmem + (static_cast<uint32_t>(quad * 32) << 16) + acc * NCOLS + (2 * qp) * HEADS;
           const float ksc = ksc_next;
-          if (OPB == 1) ksc_next = (j + 1 < U.n_kt && s + KT < p.T) ? ks_row[s + KT] : 1.f;
+          if (OPB == 1) ksc_next = (j + 1 < U.kt1 && s + KT < p.T) ? ks_row[s + KT] : 1.f;
           {
             uint32_t x[64];
             tmem_ld32_x64(ta, x);
@@ -624,6 +648,25 @@ bool stream_smem_plan(int k, int key_tile, int fp8, int* n_stages, int* pool_cap
   return false;
 }
 
+// Key partitions per unit for a launch of n_units units whose longest unit
+// spans max_kt key tiles: when the units cannot give every SM one, each
+// unit's keys are split over several CTAs (at least 4 tiles a partition).
+int stream_split_count(long long n_units, int max_kt, int n_sm) {
+  if (n_units <= 0 || n_units >= n_sm) return 1;
+  const long long by_sm = n_sm / n_units;
+  const long long by_len = max_kt / 4;
+  const long long s = std::min(by_sm, by_len);
+  return s > 1 ? static_cast<int>(s) : 1;
+}
+
+size_t stream_split_bytes_bound(int B, int S, int k, int query_chunk, int n_sm) {
+  const long long rows = query_chunk > 0 ? std::min(S, query_chunk) : S;
+  const long long units = static_cast<long long>(B) * ((rows + QT - 1) / QT);
+  if (units >= n_sm) return 0;
+  // B * part_rows * n_split <= QT * units * (n_sm / units) <= QT * n_sm
+  return static_cast<size_t>(QT) * n_sm * k * 8 + 512;
+}
+
 si_status launch_stream_topk(const void* q, const void* kc, const float* w, int B, int S, int T,
                              int H, int D, int m, int k, int32_t* out_idx, float* out_score,
                              cudaStream_t stream, const StreamConfig& cfg) {
@@ -643,9 +686,11 @@ si_status launch_stream_topk(const void* q, const void* kc, const float* w, int 
   st = encode_tmap_2d(&tm_kc, dt, kc, DIM, static_cast<uint64_t>(B) * T,
                       static_cast<uint64_t>(DIM) * opb, box_inner, KT);
   if (st != SI_OK) return st;
-  int* err = nullptr;
-  st = device_error_record(&err);
-  if (st != SI_OK) return st;
+  int* err = cfg.err;
+  if (!err) {
+    st = device_error_record(&err);
+    if (st != SI_OK) return st;
+  }
 
   int dev = 0, n_sm = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -653,8 +698,11 @@ si_status launch_stream_topk(const void* q, const void* kc, const float* w, int 
   e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
 
-  auto kern = cfg.fp8 ? stream_topk_kernel<1> : stream_topk_kernel<2>;
+  auto kern = cfg.fp8 ? stream_topk_kernel<1, false> : stream_topk_kernel<2, false>;
+  auto kern_split = cfg.fp8 ? stream_topk_kernel<1, true> : stream_topk_kernel<2, true>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(kern_split, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
 
   Params p;
@@ -679,19 +727,76 @@ si_status launch_stream_topk(const void* q, const void* kc, const float* w, int 
   // over the output; without them the managers sort before storing
   p.sort_rows = (!cfg.unsorted && out_score == nullptr) ? 1 : 0;
 
-  // chunk driver: one persistent launch per chunk of queries
+  // chunk driver: one persistent launch per chunk of queries; a chunk with
+  // fewer units than SMs splits its units' keys over CTAs (partials in
+  // scratch, then the merge kernel)
   const int n_qt_total = (S + QT - 1) / QT;
   const int chunk_qt = cfg.query_chunk > 0 ? std::max(1, cfg.query_chunk / QT) : n_qt_total;
+  auto chunk_split = [&](int qt0, int qt1) {
+    const int t_last = std::min(qt1 * QT, S) - 1;
+    const long long n = std::min<long long>((static_cast<long long>(cfg.row0) + t_last + 1) / m, T);
+    const int max_kt = static_cast<int>((n + KT - 1) / KT);
+    return cfg.allow_split ? stream_split_count(static_cast<long long>(B) * (qt1 - qt0), max_kt, n_sm) : 1;
+  };
+  size_t part_bytes = 0;
   for (int qt0 = 0; qt0 < n_qt_total; qt0 += chunk_qt) {
+    const int qt1 = std::min(n_qt_total, qt0 + chunk_qt);
+    const int ns = chunk_split(qt0, qt1);
+    if (ns > 1)
+      part_bytes = std::max(part_bytes, static_cast<size_t>(B) * (qt1 - qt0) * QT * ns * k * 8 + 256);
+  }
+  void* part_raw = nullptr;
+  uint8_t* part_base = nullptr;
+  if (part_bytes) {
+    if (cfg.split_ws && cfg.split_ws_bytes >= part_bytes) {
+      part_base = static_cast<uint8_t*>(cfg.split_ws);
+    } else {
+      st = scratch_alloc(&part_raw, part_bytes, stream, "the split-key partial top-ks");
+      if (st != SI_OK) return st;
+      part_base = static_cast<uint8_t*>(part_raw);
+    }
+    part_base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(part_base) + 255) & ~static_cast<uintptr_t>(255));
+  }
+  bool merged_sorted = true;
+  SplitParams x;
+  for (int qt0 = 0; qt0 < n_qt_total && st == SI_OK; qt0 += chunk_qt) {
     p.qt_begin = qt0;
     p.qt_end = std::min(n_qt_total, qt0 + chunk_qt);
-    const long long n_units = static_cast<long long>(B) * (p.qt_end - p.qt_begin);
-    const int grid = static_cast<int>(std::min<long long>(n_sm, n_units));
-    kern<<<grid, THREADS, smem, stream>>>(tm_q, tm_kc, p);
+    x.n_split = chunk_split(p.qt_begin, p.qt_end);
+    x.part_rows = (p.qt_end - p.qt_begin) * QT;
+    const size_t part_entries = static_cast<size_t>(B) * x.part_rows * x.n_split * k;
+    x.part_idx = x.n_split > 1 ? reinterpret_cast<int32_t*>(part_base) : nullptr;
+    x.part_score = x.n_split > 1 ? reinterpret_cast<float*>(part_base + part_entries * 4) : nullptr;
+    const long long n_work = static_cast<long long>(B) * (p.qt_end - p.qt_begin) * x.n_split;
+    const int grid = static_cast<int>(std::min<long long>(n_sm, n_work));
+    if (x.n_split > 1)
+      kern_split<<<grid, THREADS, smem, stream>>>(tm_q, tm_kc, p, x);
+    else
+      kern<<<grid, THREADS, smem, stream>>>(tm_q, tm_kc, p, x);
     e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "stream_topk_kernel launch");
+    if (e != cudaSuccess) {
+      st = cuda_fail(e, "stream_topk_kernel launch");
+      break;
+    }
+    if (x.n_split > 1) {
+      // the exact top-k of each row's partials, sorted, into the outputs
+      const int rows = std::min(x.part_rows, S - p.qt_begin * QT);
+      for (int b = 0; b < B && st == SI_OK; ++b) {
+        const size_t pb = static_cast<size_t>(b) * x.part_rows * x.n_split * k;
+        const size_t ob = (static_cast<size_t>(b) * S + p.qt_begin * QT) * k;
+        st = launch_merge_splits(x.part_idx + pb, x.part_score + pb, rows, x.n_split, k, out_idx + ob,
+                                 out_score ? out_score + ob : nullptr, stream);
+      }
+    } else {
+      merged_sorted = false;
+    }
   }
-  return SI_OK;
+  if (part_raw) {
+    e = cudaFreeAsync(part_raw, stream);
+    if (e != cudaSuccess && st == SI_OK) st = cuda_fail(e, "cudaFreeAsync");
+  }
+  if (cfg.out_sorted) *cfg.out_sorted = st == SI_OK && merged_sorted;
+  return st;
 }
 
 }  // namespace si

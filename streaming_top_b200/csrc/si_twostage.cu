@@ -580,7 +580,7 @@ size_t two_stage_workspace_bytes(int B, int S, int T, int G, int n_keep, int chu
 
 si_status launch_two_stage(const void* q, const void* kc, const float* w, int B, int S, int T, int m, int k,
                            int G, int n_keep, int chunk, int32_t* out_idx, float* out_score, void* workspace,
-                           size_t workspace_bytes, uint64_t wait_limit_ns, cudaStream_t stream) {
+                           size_t workspace_bytes, uint64_t wait_limit_ns, int* err, cudaStream_t stream) {
   const size_t need = two_stage_workspace_bytes(B, S, T, G, n_keep, chunk);
   void* raw = nullptr;
   void* ws = workspace;
@@ -588,12 +588,8 @@ si_status launch_two_stage(const void* q, const void* kc, const float* w, int B,
     if (workspace_bytes < need)
       return fail(SI_ERR_INVALID_ARGUMENT, "workspace of %zu bytes < %zu needed", workspace_bytes, need);
   } else {
-    cudaError_t e = cudaMallocAsync(&raw, need, stream);
-    if (e != cudaSuccess) {
-      cudaGetLastError();
-      return fail(SI_ERR_OUT_OF_MEMORY, "cudaMallocAsync(%zu) for the two-stage scratch: %s", need,
-                  cudaGetErrorString(e));
-    }
+    const si_status sa = scratch_alloc(&raw, need, stream, "the two-stage scratch");
+    if (sa != SI_OK) return sa;
     ws = raw;
   }
   auto carve = [](uintptr_t& cur, size_t bytes) {
@@ -612,11 +608,9 @@ si_status launch_two_stage(const void* q, const void* kc, const float* w, int B,
 
   si_status st = SI_OK;
   int dev = 0, n_sm = 0;
-  int* err = nullptr;
   cudaError_t e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) st = cuda_fail(e, "device query");
-  if (st == SI_OK) st = device_error_record(&err);
   if (st == SI_OK && nb > 0) {
     const long long n = static_cast<long long>(B) * nb * F_DIM;
     const long long grid = std::min<long long>((n + 127) / 128, static_cast<long long>(n_sm) * 16);
@@ -662,6 +656,7 @@ si_status launch_two_stage(const void* q, const void* kc, const float* w, int B,
         cfg.test_withhold = 0;
         cfg.unsorted = true;
         cfg.row0 = c0;
+        cfg.err = err;
         st = launch_stream_topk(qb, kp + static_cast<size_t>(b) * nb * F_DIM, wb, 1, R, nb, F_HEADS, F_DIM, m * G,
                                 n_keep, coarse, nullptr, stream, cfg);
         if (st != SI_OK) break;

@@ -21,6 +21,7 @@ _LIB = os.path.join(_HERE, "libsynth.so")
 _lib = None
 
 TENSOR_Q, TENSOR_KC, TENSOR_W = 1, 2, 3
+TENSOR_QA, TENSOR_KV = 4, 5  # the sparse attention's queries and compressed latents
 
 
 def build(force: bool = False) -> str:
@@ -342,3 +343,12 @@ def make_inputs_rows(wl: Workload, rows, fmt: str = "bf16", seed: int | None = N
     if qs is not None:
         full["q_scale"] = qs
     return full
+
+
+def attention_inputs(B: int, S: int, T: int, seed: int, H: int = 64, Dk: int = 576, kind: str = "gauss"):
+    """Inputs of the sparse attention over selected latents: q [B, S, H, Dk]
+    and kv [B, T, Dk] as bf16 bits, N(0, 1) (so that with scale 1/sqrt(Dk) the
+    logits have unit spread) or integers in {-3..3} (kind 'int')."""
+    q = matrix(B * S * H, Dk, seed, TENSOR_QA, kind, 1.0).reshape(B, S, H, Dk)
+    kv = matrix(B * T, Dk, seed, TENSOR_KV, kind, 1.0).reshape(B, T, Dk)
+    return q, kv

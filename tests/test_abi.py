@@ -35,6 +35,55 @@ def test_library_exports(name):
     assert hasattr(si.lib(), name), name
 
 
+def declared_prototypes():
+    """{name: (return type, [parameter types])} of every SI_API function."""
+    out = {}
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        for ret, name, params in re.findall(r"SI_API\s+([\w\s\*]+?)\s*\b(si_\w+)\s*\(([^)]*)\)", src):
+            ps = [" ".join(p.split()) for p in params.split(",")]
+            ps = [] if ps == ["void"] else ps
+            # drop the parameter name: the last identifier, unless the type is all there is
+            types = [re.sub(r"\s*\b\w+$", "", p) if re.search(r"[\w\*]\s+\w+$", p) else p for p in ps]
+            out[name] = (" ".join(ret.split()), types)
+    return out
+
+
+def _ctype_ok(c_type: str, ct) -> bool:
+    c_type = c_type.replace("const ", "")
+    if c_type == "float":
+        return ct is ctypes.c_float
+    if "*" in c_type:
+        if c_type == "char*" or c_type == "char *":
+            return ct is ctypes.c_char_p
+        return ct is ctypes.c_void_p or (isinstance(ct, type) and issubclass(ct, ctypes._Pointer))
+    return {"int": ctypes.c_int, "si_status": ctypes.c_int, "int64_t": ctypes.c_int64,
+            "size_t": ctypes.c_size_t, "unsigned long long": ctypes.c_ulonglong}[c_type] is ct
+
+
+@pytest.mark.parametrize("name", sorted(declared_prototypes()))
+def test_binding_prototypes_match_the_headers(name):
+    """The ctypes prototypes of the binding have the headers' arity and types,
+    so a change of either side is caught here rather than by a wrong call."""
+    ret, params = declared_prototypes()[name]
+    f = getattr(si.lib(), name)
+    assert f.argtypes is not None, f"{name}: the binding sets no argtypes"
+    assert len(f.argtypes) == len(params), (name, params, f.argtypes)
+    for c_type, ct in zip(params, f.argtypes):
+        assert _ctype_ok(c_type, ct), (name, c_type, ct)
+    if ret == "void":
+        assert f.restype is None, name
+    else:
+        assert _ctype_ok(ret, f.restype), (name, ret, f.restype)
+
+
+def test_options_struct_matches_the_header():
+    src = re.sub(r"/\*.*?\*/", "", open(os.path.join(ROOT, "include", "streaming_top.h")).read(), flags=re.S)
+    body = re.search(r"typedef struct si_options \{(.*?)\} si_options;", src, flags=re.S).group(1)
+    fields = [re.search(r"(\w+)\s*;", d).group(1) for d in body.split(";") if d.strip() for d in [d + ";"]]
+    assert fields == [f for f, _ in si.Options._fields_]
+
+
 def test_status_strings_and_version():
     L = si.lib()
     assert L.si_status_string(si.SI_ERR_TIMEOUT) == b"SI_ERR_TIMEOUT"
@@ -83,7 +132,12 @@ def test_fp8_needs_scales():
 
 
 def test_workspace_size():
-    assert si.workspace_size(1, 1024, 256, 64, 128, 4, 64, materialize=False) == 0
+    # enough 4-query units for any GPU: no split-key partials, no scratch
+    assert si.workspace_size(1, 8192, 2048, 64, 128, 4, 64, materialize=False) == 0
+    # few units: room for the split-key partials (a bound independent of row0)
+    small = si.workspace_size(1, 64, 1 << 16, 64, 128, 4, 64, materialize=False)
+    assert small >= 4 * 148 * 64 * 8
+    assert si.workspace_size(1, 64, 1 << 16, 64, 128, 4, 64, mxfp4=True) == small + (1 << 16) * 128 * 2 + 256
     need = si.workspace_size(1, 1024, 256, 64, 128, 4, 64, materialize=True)
     assert need >= 4 * 1024 * 256 * 65
 
@@ -121,9 +175,10 @@ def test_mxfp4_validation():
     o.workspace, o.workspace_bytes = P, 64  # too small for the decoded keys
     assert L.si_indexer_topk_ex(*args) == si.SI_ERR_INVALID_ARGUMENT
     o.workspace, o.workspace_bytes = None, 0
-    assert L.si_indexer_workspace_size(2, 64, 16, 64, 128, 4, 8, 0, ctypes.byref(o)) == 2 * 16 * 128 * 2 + 256
     o.dtype = si.SI_DTYPE_BF16
-    assert L.si_indexer_workspace_size(2, 64, 16, 64, 128, 4, 8, 0, ctypes.byref(o)) == 0
+    base = L.si_indexer_workspace_size(2, 64, 16, 64, 128, 4, 8, 0, ctypes.byref(o))
+    o.dtype = si.SI_DTYPE_MXFP4_KEYS
+    assert L.si_indexer_workspace_size(2, 64, 16, 64, 128, 4, 8, 0, ctypes.byref(o)) == base + 2 * 16 * 128 * 2 + 256
     assert L.si_mxfp4_to_bf16(P, P, 4, 48, P, None) == si.SI_ERR_INVALID_ARGUMENT  # D % 32
     assert L.si_mxfp4_to_bf16(P, P, -1, 128, P, None) == si.SI_ERR_INVALID_ARGUMENT
     assert L.si_mxfp4_to_bf16(P + 8, P, 4, 128, P, None) == si.SI_ERR_INVALID_ARGUMENT  # alignment
