@@ -48,6 +48,32 @@ def load_peaks() -> dict:
             "source": "fallback"}
 
 
+def measure_fp8_peak(dev) -> float | None:
+    """Dense e4m3 matmul throughput of this GPU (torch._scaled_mm, 8192^3,
+    bf16 output, best of 10 after 3 warm-ups, CUDA events): the denominator
+    of the e4m3 roofline.  None when the probe is unavailable."""
+    import torch
+    try:
+        n = 8192
+        a = torch.randn((n, n), device=dev).to(torch.float8_e4m3fn)
+        b = torch.randn((n, n), device=dev).to(torch.float8_e4m3fn).t()
+        one = torch.ones((), device=dev, dtype=torch.float32)
+        best = None
+        for i in range(13):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+            e1.record()
+            torch.cuda.synchronize(dev)
+            if i >= 3:
+                t = e0.elapsed_time(e1)
+                best = t if best is None else min(best, t)
+        del a, b
+        return 2.0 * n ** 3 / (best * 1e-3) / 1e12
+    except Exception:  # noqa: BLE001 -- an unavailable probe falls back to the nominal ratio
+        return None
+
+
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
     for f in ("si_stream.cu", "si_topk.cuh", "si_ptx.cuh"):
@@ -186,6 +212,43 @@ def oracle_sample(wl, inp, rows, two_stage: bool = False) -> tuple[float, int]:
     return dt, pairs
 
 
+def oracle_all_cores(wl, inp, two_stage: bool, seconds: float) -> dict:
+    """The same oracle, unchanged, on every host core: one thread per core,
+    each running the C oracle (which releases the GIL) on its own 16-row
+    groups of uniformly sampled rows, for about `seconds` of wall time."""
+    import threading
+    cores = os.cpu_count() or 1
+    rows = synth.sample_rows(16 * 64 * cores, wl.m * 4, wl.S, seed=wl.seed + 98)
+    np.random.default_rng(wl.seed).shuffle(rows)
+    lock = threading.Lock()
+    state = {"next": 0, "pairs": 0, "rows": 0}
+    t_end = time.perf_counter() + seconds
+
+    def worker():
+        while time.perf_counter() < t_end:
+            with lock:
+                i = state["next"]
+                state["next"] += 16
+            if i >= len(rows):
+                return
+            _, pr = oracle_sample(wl, inp, np.sort(rows[i:i + 16]), two_stage)
+            with lock:
+                state["pairs"] += pr
+                state["rows"] += 16
+
+    t0 = time.perf_counter()
+    threads = [threading.Thread(target=worker) for _ in range(cores)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+    dt = time.perf_counter() - t0
+    return {"value": state["pairs"] / dt, "unit": "pairs/s", "cores": cores, "kind": "oracle",
+            "sample": f"{state['rows']} uniformly sampled query rows of the {wl.name} workload ({state['pairs']} "
+                      f"visible pairs, {dt:.1f} s wall), the C oracle unchanged on {cores} threads, one per "
+                      "host core, fp64, full sort"}
+
+
 def run_reference(args, wl):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -221,6 +284,132 @@ def run_reference(args, wl):
     }
     print(json.dumps(line))
     return 0
+
+
+# ------------------------------------------------------- million-token record
+def million_record(args, dev, sampler_index: int) -> dict:
+    """The million-token workload (B=1, S=1,048,576, T=262,144, k=512, planted
+    inputs, seed 4) beside the headline: one streaming call per format (bf16,
+    e4m3 with per-row scales) with all inputs resident, W=1 + K=2 timed calls,
+    and the bf16 call once more end to end through si_indexer_topk_host (host
+    buffers, query chunks streamed through the device).  Peak HBM is the
+    path's own device memory: inputs, outputs and library scratch."""
+    import torch
+
+    import streaming_top_b200 as si
+    wl = synth.WORKLOADS["million"]
+    B, S, T, H, D, k = wl.B, wl.S, wl.T, wl.H, wl.D, wl.k
+    P = wl.visible_pairs()
+    flop = P * 2 * H * D
+    peaks = load_peaks()
+    fp8_peak = measure_fp8_peak(dev)
+    out = {"workload": f"million: B={B}, S={S}, m={wl.m} (T={T}), H_I={H}, D={D}, k={k}, planted inputs, "
+                       f"seed {wl.seed}", "visible_pairs": P, "calls": "1 warm-up + 2 timed per format"}
+    stream = torch.cuda.current_stream(dev)
+    chunk = 16384
+    # bf16 q in page-locked host memory (also the host-buffer call's input)
+    hq = torch.empty((B, S, H, D), dtype=torch.int16).pin_memory()
+    hqn = hq.numpy().view(np.uint16)
+    for t0 in range(0, S, chunk):
+        synth.q_rows(wl, 0, t0, min(chunk, S - t0), "bf16", out=hqn[0, t0:t0 + chunk])
+    for fmt in ("bf16", "e4m3"):
+        rest = synth.make_inputs(wl, fmt=fmt, skip_q=True)
+        torch.cuda.synchronize(dev)
+        torch.cuda.empty_cache()
+        base_mem = torch.cuda.memory_allocated(dev)
+        torch.cuda.reset_peak_memory_stats(dev)
+        if fmt == "bf16":
+            q = hq.to(dev, non_blocking=True).view(torch.bfloat16)
+            kc = torch.from_numpy(rest["kc"].view(np.int16)).view(torch.bfloat16).to(dev)
+            qs = ks = None
+        else:
+            q = torch.empty((B, S, H, D), dtype=torch.uint8, device=dev)
+            qs = torch.empty((B, S, H), dtype=torch.float32, device=dev)
+            buf = torch.empty((chunk, H, D), dtype=torch.uint8).pin_memory()
+            sbuf = torch.empty((chunk, H), dtype=torch.float32).pin_memory()
+            for t0 in range(0, S, chunk):
+                n = min(chunk, S - t0)
+                torch.cuda.synchronize(dev)
+                synth.q_rows(wl, 0, t0, n, "e4m3", out=buf.numpy()[:n], scale_out=sbuf.numpy()[:n])
+                q[0, t0:t0 + n].copy_(buf[:n], non_blocking=True)
+                qs[0, t0:t0 + n].copy_(sbuf[:n], non_blocking=True)
+            kc = torch.from_numpy(rest["kc"]).to(dev)
+            ks = torch.from_numpy(rest["kc_scale"]).to(dev)
+        w = torch.from_numpy(rest["w"]).to(dev)
+        oi = torch.empty((B, S, k), dtype=torch.int32, device=dev)
+        osc = torch.empty((B, S, k), dtype=torch.float32, device=dev)
+        torch.cuda.synchronize(dev)
+        path_bytes = sum(t.numel() * t.element_size() for t in (q, qs, kc, ks, w, oi, osc) if t is not None)
+
+        def call(mid=None):
+            si.indexer_topk(q, kc, w, wl.m, k, q_scale=qs, kc_scale=ks, out_idx=oi, out_score=osc, unsorted=True,
+                            stream=stream)
+            if mid is not None:
+                mid.record(stream)
+            si.sort_topk_rows(oi, osc, stream=stream)
+
+        call()
+        sampler = ClockSampler(sampler_index)
+        sampler.start()
+        time.sleep(0.3)
+        evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(2)]
+        for e0, em, e1 in evs:
+            e0.record(stream)
+            call(em)
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        clocks = sampler.stop()
+        if si.device_status(stream) != si.SI_OK:
+            raise RuntimeError(f"device error in the million-token {fmt} calls")
+        ms = sum(a.elapsed_time(b) for a, _, b in evs) / len(evs)
+        ms_k = sum(a.elapsed_time(b) for a, b, _ in evs) / len(evs)
+        if fmt == "e4m3" and fp8_peak:
+            peak_tc, peak_src = fp8_peak, "measured in this run: torch._scaled_mm e4m3 8192^3, burst"
+        else:
+            peak_tc = peaks["bf16_tflops"] * (2.0 if fmt == "e4m3" else 1.0)
+            peak_src = (f"{peaks['source']} bf16 dense matmul, burst" +
+                        (" x2 (nominal fp8 / bf16 dense ratio)" if fmt == "e4m3" else ""))
+        rec = {"ms_per_call": ms, "kernel_ms": ms_k, "pairs_per_s": P / (ms * 1e-3),
+               "tflops": flop / (ms * 1e-3) / 1e12,
+               "frac_peak": flop / (ms * 1e-3) / 1e12 / peak_tc,
+               "kernel_frac_peak": flop / (ms_k * 1e-3) / 1e12 / peak_tc,
+               "peak": peak_tc, "peak_source": peak_src,
+               "peak_hbm_gb": (torch.cuda.max_memory_allocated(dev) - base_mem) / 1e9,
+               "hbm_breakdown_gb": {"q": (q.numel() * q.element_size() + (qs.numel() * 4 if qs is not None else 0))
+                                    / 1e9, "kc": kc.numel() * kc.element_size() / 1e9, "w": w.numel() * 4 / 1e9,
+                                    "out_idx + out_score": 2 * oi.numel() * 4 / 1e9, "library_workspace": 0.0},
+               "path_bytes_gb": path_bytes / 1e9, "clocks": clocks}
+        out[fmt] = rec
+        del q, qs, kc, ks, w, oi, osc
+        torch.cuda.empty_cache()
+    # the same bf16 workload end to end from host buffers: only the keys and
+    # two chunks of query rows are ever on the device
+    rest = synth.make_inputs(wl, fmt="bf16", skip_q=True)
+    hk = torch.from_numpy(rest["kc"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    hw = torch.from_numpy(rest["w"]).pin_memory()
+    hqb = hq.view(torch.bfloat16)
+    h_idx = torch.empty((B, S, k), dtype=torch.int32).pin_memory()
+    h_sc = torch.empty((B, S, k), dtype=torch.float32).pin_memory()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    si.indexer_topk_host(hqb, hk, hw, wl.m, k, out_idx=h_idx, out_score=h_sc, stream=stream, device=dev)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    dev_bytes = si.indexer_topk_host_workspace_size(B, S, T, H, D, k)
+    out["bf16_host_streamed"] = {
+        "api": "si_indexer_topk_host (C ABI): host q, kc, w in, host results out; 8192-row query chunks through "
+               "two device slots, copies overlapped with the scoring",
+        "ms_per_call": e0.elapsed_time(e1), "pairs_per_s": P / (e0.elapsed_time(e1) * 1e-3),
+        "peak_hbm_gb": dev_bytes / 1e9,
+        "h2d_bytes": hq.numel() * 2 + hk.numel() * 2 + hw.numel() * 4, "d2h_bytes": 2 * B * S * k * 4,
+        "calls": "1 (after the device-resident calls)"}
+    out["pages_context"] = ("StreamIndex (abstract) reports 6.21 GB peak at S=1,048,576 on one H200 for the indexer "
+                            "step, without saying how q is held; here the resident path holds q (16 GiB bf16), all "
+                            "outputs (4 GiB) and no scratch, the host-streamed path only the keys and two query "
+                            "chunks")
+    del hq, hqn, hk, hw, h_idx, h_sc
+    return out
 
 
 # ------------------------------------------------------------------ CUDA path
@@ -275,6 +464,14 @@ def run_ours(args, wl):
     kms = torch.from_numpy(inp["kc_mx_scale"]).to(dev) if mx else None
     out_idx = torch.empty((wl.B, rows_here, wl.k), dtype=torch.int32, device=dev)
     out_score = torch.empty((wl.B, rows_here, wl.k), dtype=torch.float32, device=dev)
+    # library scratch, allocated here so that torch's peak counts it
+    if two:
+        ws_bytes = si.two_stage_workspace_size(wl.B, wl.S, wl.T, query_chunk=TWO_STAGE_CHUNK, **TWO_STAGE)
+    elif mx:
+        ws_bytes = si.workspace_size(wl.B, rows_here, wl.T, wl.H, wl.D, wl.m, wl.k, mxfp4=True)
+    else:
+        ws_bytes = 0
+    workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev) if ws_bytes else None
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)  # > 126 MB L2
     stream = torch.cuda.current_stream(dev)
     torch.cuda.synchronize(dev)
@@ -287,16 +484,17 @@ def run_ours(args, wl):
         if two:
             # one si_indexer_topk_two_stage call (pool, coarse, fine, select, row sort)
             si.indexer_topk_two_stage(q, kc, w, wl.m, wl.k, query_chunk=TWO_STAGE_CHUNK, out_idx=out_idx,
-                                      out_score=out_score, stream=stream, **TWO_STAGE)
+                                      out_score=out_score, stream=stream, workspace=workspace, **TWO_STAGE)
             if mid is not None:
                 mid.record(stream)
             return
         if rows_mode:
             si.indexer_topk_rows(q, kc, w, wl.m, wl.k, r0, q_scale=qs, kc_scale=ks, out_idx=out_idx,
-                                 out_score=out_score, unsorted=True, stream=stream, kc_mx_scale=kms)
+                                 out_score=out_score, unsorted=True, stream=stream, kc_mx_scale=kms,
+                                 workspace=workspace)
         else:
             si.indexer_topk(q, kc, w, wl.m, wl.k, q_scale=qs, kc_scale=ks, out_idx=out_idx,
-                            out_score=out_score, unsorted=True, stream=stream, kc_mx_scale=kms)
+                            out_score=out_score, unsorted=True, stream=stream, kc_mx_scale=kms, workspace=workspace)
         if mid is not None:
             mid.record(stream)
         si.sort_topk_rows(out_idx, out_score, stream=stream)
@@ -339,16 +537,28 @@ def run_ours(args, wl):
         ms_kernel = max_over_ranks(ms_kernel, dev)
         ms_sort = max_over_ranks(ms_sort, dev)
 
-    # end to end through the host-buffer API: H2D inputs, kernel, D2H results
+    # end to end through the C ABI's host-buffer entry point (si_indexer_topk_host):
+    # page-locked host inputs in, host results out, the copies of the query
+    # chunks overlapped with the scoring inside the call
     hq, hk, hw = (host_tensor(n).pin_memory() for n in ("q", "kc", "w"))
     hqs = torch.from_numpy(inp["q_scale"]).pin_memory() if fp8 else None
     hks = torch.from_numpy(inp["kc_scale"]).pin_memory() if fp8 else None
     hkms = torch.from_numpy(inp["kc_mx_scale"]).pin_memory() if mx else None
+    h_idx = torch.empty((wl.B, rows_here, wl.k), dtype=torch.int32).pin_memory()
+    h_score = torch.empty((wl.B, rows_here, wl.k), dtype=torch.float32).pin_memory()
     bufs = {}
+
+    def e2e_step():
+        if two:
+            si.indexer_topk_two_stage_host(hq, hk, hw, wl.m, wl.k, device=dev, bufs=bufs,
+                                           query_chunk=TWO_STAGE_CHUNK, **TWO_STAGE)
+        else:
+            si.indexer_topk_host(hq, hk, hw, wl.m, wl.k, q_scale=hqs, kc_scale=hks, kc_mx_scale=hkms,
+                                 row0=r0 or 0, out_idx=h_idx, out_score=h_score, stream=stream, device=dev)
+
     for _ in range(max(1, args.warmup)):
-        si.indexer_topk_host(hq, hk, hw, wl.m, wl.k, q_scale=hqs, kc_scale=hks, device=dev, bufs=bufs,
-                             row0=r0, kc_mx_scale=hkms, two_stage=TWO_STAGE if two else None,
-                             query_chunk=TWO_STAGE_CHUNK if two else 0)
+        e2e_step()
+    e2e_dev = torch.cuda.memory_allocated(dev)
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
     if world > 1:
@@ -356,9 +566,7 @@ def run_ours(args, wl):
     torch.cuda.synchronize(dev)
     for e0, e1 in e2e_ev:
         e0.record(stream)
-        si.indexer_topk_host(hq, hk, hw, wl.m, wl.k, q_scale=hqs, kc_scale=hks, device=dev, bufs=bufs,
-                             sync=False, row0=r0, kc_mx_scale=hkms, two_stage=TWO_STAGE if two else None,
-                             query_chunk=TWO_STAGE_CHUNK if two else 0)
+        e2e_step()
         e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev) / args.steps
@@ -369,7 +577,17 @@ def run_ours(args, wl):
 
     h2d = nbytes(hq, hk, hw, hqs, hks, hkms)
     d2h = out_idx.numel() * 4 + out_score.numel() * 4
-    del bufs
+    # device memory of the host-buffer call: the keys and two chunks of rows
+    e2e_device_bytes = (si.two_stage_workspace_size(wl.B, rows_here, wl.T, **TWO_STAGE,
+                                                    query_chunk=TWO_STAGE_CHUNK) + nbytes(q, kc, w, out_idx, out_score)
+                        if two else si.indexer_topk_host_workspace_size(
+                            wl.B, rows_here, wl.T, wl.H, wl.D, wl.k,
+                            dtype=si.SI_DTYPE_FP8_E4M3 if fp8 else (si.SI_DTYPE_MXFP4_KEYS if mx else si.SI_DTYPE_BF16)))
+    del bufs, e2e_dev
+
+    million = None
+    if world == 1 and wl.name == "v4flash" and args.fmt == "bf16" and not two and not args.no_million:
+        million = million_record(args, dev, sampler.idx)
 
     if world > 1:
         dist.barrier()
@@ -398,11 +616,16 @@ def run_ours(args, wl):
     alg_bytes = nbytes(q, kc, w, out_idx, out_score, qs, ks, kms)
     # the committed DRAM capture is of the whole-sequence bf16 launch
     traffic = None if fp8 or mx or two or (rows_mode and world > 1) else ncu_traffic(wl.name)
-    # a contraction is measured against the peak of its own type: fp8 takes the
-    # measured bf16 matmul peak times the nominal fp8 / bf16 ratio (4.5 / 2.25)
-    peak_tc = peaks["bf16_tflops"] * (2.0 if fp8 else 1.0)
-    peak_src = (f"{peaks['source']} bf16 dense matmul, burst" +
-                (", x2 (nominal fp8 / bf16 dense ratio)" if fp8 else ""))
+    # a contraction is measured against the peak of its own type: fp8 takes a
+    # dense e4m3 matmul measured in this run (else the measured bf16 peak times
+    # the nominal fp8 / bf16 ratio, 4.5 / 2.25)
+    fp8_peak = measure_fp8_peak(dev) if fp8 else None
+    if fp8 and fp8_peak:
+        peak_tc, peak_src = fp8_peak, "measured in this run: torch._scaled_mm e4m3 8192^3, burst"
+    else:
+        peak_tc = peaks["bf16_tflops"] * (2.0 if fp8 else 1.0)
+        peak_src = (f"{peaks['source']} bf16 dense matmul, burst" +
+                    (", x2 (nominal fp8 / bf16 dense ratio)" if fp8 else ""))
     cpu = None
     if world == 1 and args.cpu_seconds > 0:
         rows = synth.sample_rows(4096, wl.m * 4, wl.S, seed=wl.seed + 99)
@@ -418,6 +641,7 @@ def run_ours(args, wl):
         cpu = {"value": p_tot / t_tot, "unit": "pairs/s", "cores": 1, "kind": "oracle",
                "sample": f"{done} uniformly sampled query rows of the {wl.name} workload ({p_tot} visible "
                          f"pairs, {t_tot:.1f} s), single-threaded C oracle, fp64, full sort"}
+        cpu["all_cores"] = oracle_all_cores(wl, inp, two, seconds=min(args.cpu_seconds, 10.0))
     line = {
         "metric": METRIC, "value": value, "unit": "pairs/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
@@ -436,11 +660,13 @@ def run_ours(args, wl):
         "frac_bf16_peak_sustained": tflops / peaks["bf16_tflops_sustained"] if peaks["bf16_tflops_sustained"] else None,
         "hbm_gbs": alg_bytes / (ms_step * 1e-3) / 1e9,
         "frac_hbm": alg_bytes / (ms_step * 1e-3) / 1e9 / peaks["hbm_gbs"],
-        "peak_hbm_gb": peak_mem / 1e9,
+        # the path's own device memory: inputs, outputs and library scratch
+        # (torch's peak less the bench's L2-flush buffer, which is no part of it)
+        "peak_hbm_gb": (peak_mem - flush.numel()) / 1e9,
         "hbm_breakdown_gb": {"q": nbytes(q, qs) / 1e9, "kc": nbytes(kc, ks, kms) / 1e9, "w": nbytes(w) / 1e9,
                              "out_idx": nbytes(out_idx) / 1e9, "out_score": nbytes(out_score) / 1e9,
-                             "l2_flush_buffer": flush.numel() / 1e9,
-                             "library_workspace": (wl.B * wl.T * wl.D * 2 + 256) / 1e9 if mx else 0.0},
+                             "library_workspace": ws_bytes / 1e9,
+                             "bench_l2_flush_buffer (not counted)": flush.numel() / 1e9},
         "kernel_ms": ({"indexer_topk_two_stage call": ms_kernel} if two else
                       {"stream_topk_kernel": ms_kernel, "row_sort_kernel": ms_sort}),
         "roofline": {"bound": "tensor",
@@ -453,10 +679,94 @@ def run_ours(args, wl):
                      "traffic": traffic, "algorithmic_bytes": alg_bytes},
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "pairs/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                "api": ("indexer_topk_two_stage on device copies (Python)" if two else
+                        "si_indexer_topk_host (C ABI, host buffers; query chunks of 8192 rows through two "
+                        "device slots, copies overlapped with the scoring)"),
+                "device_gb": e2e_device_bytes / 1e9},
         "gpu_launches": ((2 + 3 * wl.B * -(-wl.S // TWO_STAGE_CHUNK)) if two else 2) * args.steps,
         "clocks": clocks,
         "wall_s_timed": wall,
+    }
+    if million is not None:
+        line["million"] = million
+    print(json.dumps(line))
+    return 0
+
+
+# ------------------------------------------------------------ sparse attention
+ATTN_H, ATTN_DK, ATTN_DV = 64, 576, 512
+
+
+def run_attention(args, wl):
+    """One step = one si_sparse_attention call over the workload's queries:
+    every query's 64 heads attend over the 512 latents its indexer top-k
+    selected (the indexer runs once, untimed, on the workload's own planted
+    inputs).  Latents [T, 576] and attention queries [S, 64, 576] are N(0, 1)
+    bf16; out [S, 64, 512] bf16 and lse [S, 64] fp32."""
+    import torch
+
+    import streaming_top_b200 as si
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    inp = synth.make_inputs(wl)
+    qi = torch.from_numpy(inp["q"].view(np.int16)).view(torch.bfloat16).to(dev)
+    kc = torch.from_numpy(inp["kc"].view(np.int16)).view(torch.bfloat16).to(dev)
+    idx, _ = si.indexer_topk(qi, kc, torch.from_numpy(inp["w"]).to(dev), wl.m, wl.k)
+    del qi, kc
+    q, kv = synth.attention_inputs(wl.B, wl.S, wl.T, seed=wl.seed + 500)
+    qd = torch.from_numpy(q.view(np.int16)).view(torch.bfloat16).to(dev)
+    kvd = torch.from_numpy(kv.view(np.int16)).view(torch.bfloat16).to(dev)
+    del q, kv
+    out = torch.empty((wl.B, wl.S, ATTN_H, ATTN_DV), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((wl.B, wl.S, ATTN_H), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        flush.zero_()
+        si.sparse_attention(qd, kvd, idx, out=out, lse=lse, stream=stream)
+    if si.device_status(stream) != si.SI_OK:
+        raise RuntimeError("device error during warm-up")
+    sampler = ClockSampler(0 if "CUDA_VISIBLE_DEVICES" not in os.environ else
+                           int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[0]))
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    time.sleep(0.3)
+    for e0, e1 in evs:
+        flush.zero_()
+        e0.record(stream)
+        si.sparse_attention(qd, kvd, idx, out=out, lse=lse, stream=stream)
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    if si.device_status(stream) != si.SI_OK:
+        raise RuntimeError("device error during the timed steps")
+    ms = sum(a.elapsed_time(b) for a, b in evs) / len(evs)
+    nq = wl.B * wl.S
+    sel = int((idx >= 0).sum())
+    flop = 2 * ATTN_H * sel * (ATTN_DK + ATTN_DV)   # selected entries only
+    alg_bytes = sum(t.numel() * t.element_size() for t in (qd, out, lse, idx)) + kvd.numel() * 2
+    gathered = sel * (ATTN_DK + ATTN_DV) * 2
+    peaks = load_peaks()
+    line = {
+        "metric": "sparse attention over the indexer's selected latents: queries/s (TFLOP/s, % bf16 TC peak)",
+        "value": nq / (ms * 1e-3), "unit": "queries/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": f"sparse attention at the {wl.name} shape: B={wl.B}, S={wl.S} queries x 64 heads, "
+                               f"T={wl.T} latents of 576 (values: the first 512), the indexer's top-{wl.k} "
+                               f"of the planted inputs (seed {wl.seed}) as the selection",
+                   "selected_entries": sel, "l2": "q (4.8 GB) > L2, and L2 flushed before each timed step"},
+        "tflops": flop / (ms * 1e-3) / 1e12,
+        "roofline": {"bound": "tensor", "kernel": "sparse_attn_kernel", "achieved": flop / (ms * 1e-3) / 1e12,
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": flop / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                     "peak_source": f"{peaks['source']} bf16 dense matmul, burst", "traffic": None,
+                     "algorithmic_bytes": alg_bytes, "gathered_latent_bytes_from_l2": gathered},
+        "hbm_gbs": alg_bytes / (ms * 1e-3) / 1e9,
+        "gpu_launches": args.steps,
+        "clocks": clocks,
     }
     print(json.dumps(line))
     return 0
@@ -474,7 +784,9 @@ def main() -> int:
                     help="input format: bf16 (default), fp8 e4m3 with per-row scales, or mxfp4 keys "
                          "(E2M1 + E8M0 per 32 values) with bf16 queries")
     ap.add_argument("--ref-rows", type=int, default=32)
-    ap.add_argument("--method", default="one-stage", choices=["one-stage", "two-stage"],
+    ap.add_argument("--no-million", action="store_true",
+                    help="leave out the million-token record the default run adds beside the headline")
+    ap.add_argument("--method", default="one-stage", choices=["one-stage", "two-stage", "sparse-attention"],
                     help="one-stage (the streaming top-k over all visible keys) or the two-stage indexer "
                          "(2048 blocks of 8 kept by their pooled key, then the top-k of their keys)")
     ap.add_argument("--shard", default="seq", choices=["seq", "rows"],
@@ -484,6 +796,10 @@ def main() -> int:
     if args.method == "two-stage" and (args.fmt != "bf16" or args.shard == "rows"):
         raise SystemExit("--method two-stage runs bf16 inputs over whole sequences")
     wl = synth.WORKLOADS[args.workload]
+    if args.method == "sparse-attention":
+        if args.impl == "reference" or args.gpus != 1:
+            raise SystemExit("--method sparse-attention times the CUDA kernel on one GPU")
+        return run_attention(args, wl)
     if args.impl == "reference":
         return run_reference(args, wl)
     return run_ours(args, wl)
