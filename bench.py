@@ -398,7 +398,7 @@ def million_record(args, dev, sampler_index: int) -> dict:
     torch.cuda.synchronize(dev)
     dev_bytes = si.indexer_topk_host_workspace_size(B, S, T, H, D, k)
     out["bf16_host_streamed"] = {
-        "api": "si_indexer_topk_host (C ABI): host q, kc, w in, host results out; 8192-row query chunks through "
+        "api": "si_indexer_topk_host (C ABI): host q, kc, w in, host results out; 4096-row query chunks through "
                "two device slots, copies overlapped with the scoring",
         "ms_per_call": e0.elapsed_time(e1), "pairs_per_s": P / (e0.elapsed_time(e1) * 1e-3),
         "peak_hbm_gb": dev_bytes / 1e9,
@@ -681,7 +681,7 @@ def run_ours(args, wl):
         "e2e": {"value": e2e_value, "unit": "pairs/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "api": ("indexer_topk_two_stage on device copies (Python)" if two else
-                        "si_indexer_topk_host (C ABI, host buffers; query chunks of 8192 rows through two "
+                        "si_indexer_topk_host (C ABI, host buffers; query chunks of 4096 rows through two "
                         "device slots, copies overlapped with the scoring)"),
                 "device_gb": e2e_device_bytes / 1e9},
         "gpu_launches": ((2 + 3 * wl.B * -(-wl.S // TWO_STAGE_CHUNK)) if two else 2) * args.steps,

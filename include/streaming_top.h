@@ -140,7 +140,7 @@ SI_API si_status si_indexer_topk_rows(const void* q, const void* kc, const float
  * The pages stream the queries in chunks so that only one chunk is resident
  * (StreamIndex abstract, the memory bound at a million tokens); this call
  * does so from host memory: the keys are copied once, then chunks of
- * opt->query_chunk rows (0 = 8192; a multiple of 4) go through two device
+ * opt->query_chunk rows (0 = 4096; a multiple of 4) go through two device
  * slots, the copy of the next chunk in and of the previous chunk's results
  * out overlapping the scoring of the current one (two internal copy streams
  * ordered against `stream` by events).  Device memory: the keys plus two

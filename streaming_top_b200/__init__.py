@@ -377,7 +377,7 @@ def indexer_topk_host(q, kc, w, m: int, k: int, *, q_scale=None, kc_scale=None, 
     """End to end on HOST tensors (``si_indexer_topk_host``): q [B, R, H_I, D],
     w [B, R, H_I], kc [B, T, D] (and the fp8 / MXFP4 scales) in host memory,
     page-locked for the copies to overlap the scoring.  The library copies the
-    keys once and the query rows in chunks of `query_chunk` rows (0 = 8192)
+    keys once and the query rows in chunks of `query_chunk` rows (0 = 4096)
     through two device slots, overlapping the copies with the scoring, and
     returns when (idx, score) [B, R, k] are in host memory.  With `row0` the
     rows are rows row0 .. row0+R-1 of the sequences (default 0: the whole

@@ -12,8 +12,8 @@
 //
 // One CTA per SM, persistent over queries.  Per query:
 //   QK   S^T[e, h] = sum_d kv[sel[e], d] * q[h, d]: tcgen05 kind::f16, A = 128
-//        gathered latent rows (M = entries) x 64 dims per stage, SW128
-//        K-major; B = q[t] (N = 64 heads, K = 576) TMA-loaded once; fp32 into
+//        gathered latent rows (M = entries) x 64 dims per stage (TMA gather4),
+//        SW128 K-major; B = q[t] (N = 64 heads, K = 576) TMA-loaded once; fp32 into
 //        TMEM columns [64 j, 64 j + 64) for entry tile j.
 //   soft max and sum per head over the k entries (4 softmax warps, lane =
 //        entry, 32 heads at a time), P = exp(scale (s - max)) rounded to bf16
@@ -24,8 +24,9 @@
 //        per stage), B = P^T; fp32 into TMEM columns [256 + 64 v, ...) for dv
 //        tile v.
 //   out  O[t, h, dv] = O^T * (1 / sum_h), bf16; lse[t, h] fp32.
-// Warps: 0 q loads (TMA), 1 MMA issue, 2-3 gather producers (16-byte
-// cp.async into the swizzled stages), 4-7 softmax and epilogue.  Every wait
+// Warps: 0 q loads (TMA), 1 MMA issue, 2 gather producer (TMA gather4: four
+// latent rows a lane, a 16 KB stage a warp instruction), 3 idle, 4-7 softmax
+// and epilogue.  Every wait
 // is bounded; on expiry the kernel records SI_ERR_TIMEOUT, drains its copies
 // and MMAs and exits.
 #include <cuda.h>
@@ -70,10 +71,19 @@ struct ACtrl {
   int abort;
   float red[4][A_H];      // per-quadrant partial max / sum
   float head_max[A_H], head_inv[A_H];  // per head: max logit, 1 / sum of the rounded weights
+  alignas(16) int sel[A_KMAX];  // the producer's copy of the current query's selection: latent rows
 };
 
-__device__ __forceinline__ void cp16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+// TMA gather of four rows r0..r3 of a 2-D tensor map (box: 64 elements x 1
+// row), columns x .. x+63, into four consecutive 128-byte rows at dst
+// (swizzled by the map), completing `bytes` on the mbarrier.  No multicast.
+__device__ __forceinline__ void tma_gather4(void* dst, const void* tmap, uint64_t* bar, int32_t x, int32_t r0,
+                                            int32_t r1, int32_t r2, int32_t r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar)), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+      : "memory");
 }
 
 // Shared-memory descriptor of an MN-major operand with the 128-byte swizzle:
@@ -97,7 +107,8 @@ __device__ __forceinline__ void attn_error(const AttnParams& p, volatile int* ab
 }
 
 __global__ void __launch_bounds__(A_THREADS, 1)
-    sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const AttnParams p) {
+    sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
+                       const AttnParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* q_s = smem;
@@ -111,7 +122,7 @@ __global__ void __launch_bounds__(A_THREADS, 1)
   const int qk_stages = n_et * A_KB, pv_stages = 4 * n_kc;
   if (threadIdx.x == 0) {
     for (int s = 0; s < A_NS; ++s) {
-      mbar_init(&C->full[s], 64);
+      mbar_init(&C->full[s], 1);
       mbar_init(&C->empty[s], 1);
     }
     mbar_init(&C->q_full, 1);
@@ -124,7 +135,10 @@ __global__ void __launch_bounds__(A_THREADS, 1)
     *abort = 0;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) prefetch_tmap(&tm_q);
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_kv);
+  }
   if (warp == 1) tmem_alloc(&C->tmem_slot, 512);
   tc_fence_before();
   __syncthreads();
@@ -218,64 +232,64 @@ __global__ void __launch_bounds__(A_THREADS, 1)
       mma_commit(&C->done);
       if (!mbar_wait_timed(&C->done, 0, p.wait_limit_ns)) attn_error(p, abort, AERR_DRAIN);
     }
-  } else if (warp < 4) {
-    // ------------------------------------------------------------ gather producers
-    const int pt = threadIdx.x - 64;
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ gather producer (TMA gather4)
+    // The warp copies the query's selection into shared memory, then fills
+    // each 16 KB stage with one gather4 per lane: 4 latent rows x 64 dims
+    // (512 B) each, landing in the 128-byte-swizzled layout the MMA reads.
+    // One warp instruction issues the whole stage; lane 0 owns the barriers.
     uint32_t stage = 0, phase = 0;
-    int pend[3], np = 0;
+    uint32_t any_load = 0, last_par = 0;  // per stage: loaded at all / parity of the last load
     bool stop = false;
     for (int t = q0; t < nq && !stop; t += qstep) {
-      const int b = t / p.S;
-      const int32_t* sel = p.idx + static_cast<size_t>(t) * p.k;
-      const uint8_t* kvb = p.kv + static_cast<size_t>(b) * p.T * (A_DK * 2);
+      const int row_base = (t / p.S) * p.T;  // the sequence's first latent row in the tensor map
+      __syncwarp();  // every lane has issued its loads of the last query
+      for (int e = lane; e < p.k; e += 32) {
+        const int key = p.idx[static_cast<size_t>(t) * p.k + e];
+        C->sel[e] = row_base + (key >= 0 && key < p.T ? key : 0);  // padding reads row 0; its weight is 0
+      }
+      __syncwarp();
       for (int j = 0; j < qk_stages + pv_stages; ++j) {
-        const bool got = mbar_wait_bounded(&C->empty[stage], phase ^ 1u, abort, p.wait_limit_ns);
-        if (!__all_sync(0xFFFFFFFFu, got)) {
-          if (lane == 0) attn_error(p, abort, AERR_STAGE_FREE);
+        bool got = true;
+        if (lane == 0) {
+          got = mbar_wait_bounded(&C->empty[stage], phase ^ 1u, abort, p.wait_limit_ns);
+          if (got)
+            mbar_arrive_expect_tx(&C->full[stage], A_STAGE);
+          else
+            attn_error(p, abort, AERR_STAGE_FREE);
+        }
+        if (__shfl_sync(0xFFFFFFFFu, got ? 1 : 0, 0) == 0) {
           stop = true;
           break;
         }
-        const uint32_t base = smem_u32(st_s + stage * A_STAGE);
-#pragma unroll 4
-        for (int i = 0; i < 16; ++i) {
-          const int id = pt + 64 * i, ch = id & 7;
-          int row, e, col_bytes, a = 0;
-          if (j < qk_stages) {             // entry tile j / 9, K-block j % 9: 128 rows x 128 B
-            row = id >> 3;
-            e = (j / A_KB) * 128 + row;
-            col_bytes = (j % A_KB) * 128;
-          } else {                         // dv tile, 64-entry chunk: 2 atoms (64 dv each) x 64 rows x 128 B
-            const int jj = j - qk_stages;
-            a = id >> 9;
-            row = (id >> 3) & 63;
-            e = (jj % n_kc) * 64 + row;
-            col_bytes = ((jj / n_kc) * 128 + a * 64) * 2;
-          }
-          int key = sel[e];
-          key = key >= 0 && key < p.T ? key : 0;  // padding reads row 0; its weight is 0
-          cp16(base + a * 8192 + row * 128 + ((ch ^ (row & 7)) << 4),
-               kvb + static_cast<size_t>(key) * (A_DK * 2) + col_bytes + ch * 16);
+        __syncwarp();
+        int e, x, off;
+        if (j < qk_stages) {  // entry tile j / 9, K-block j % 9: 128 rows x 128 B
+          e = (j / A_KB) * 128 + 4 * lane;
+          x = (j % A_KB) * 64;
+          off = lane * 512;
+        } else {  // dv tile, 64-entry chunk: two atoms (64 dv each) of 64 rows x 128 B
+          const int jj = j - qk_stages, a = lane >> 4;
+          e = (jj % n_kc) * 64 + 4 * (lane & 15);
+          x = (jj / n_kc) * 128 + a * 64;
+          off = a * 8192 + (lane & 15) * 512;
         }
-        asm volatile("cp.async.commit_group;" ::: "memory");
-        pend[np++] = static_cast<int>(stage);
-        if (np == 3) {
-          asm volatile("cp.async.wait_group 2;" ::: "memory");
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          mbar_arrive(&C->full[pend[0]]);
-          pend[0] = pend[1];
-          pend[1] = pend[2];
-          np = 2;
-        }
+        const int4 r = *reinterpret_cast<const int4*>(&C->sel[e]);
+        tma_gather4(st_s + stage * A_STAGE + off, &tm_kv, &C->full[stage], x, r.x, r.y, r.z, r.w);
+        any_load |= 1u << stage;
+        last_par = (last_par & ~(1u << stage)) | (phase << stage);
         if (++stage == A_NS) {
           stage = 0;
           phase ^= 1u;
         }
       }
     }
-    asm volatile("cp.async.wait_group 0;" ::: "memory");
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    for (int e = 0; e < np; ++e) mbar_arrive(&C->full[pend[e]]);
-  } else {
+    // every load issued has landed before the CTA can exit
+    if (lane == 0)
+      for (int s = 0; s < A_NS; ++s)
+        if (((any_load >> s) & 1u) && !mbar_wait_timed(&C->full[s], (last_par >> s) & 1u, p.wait_limit_ns))
+          attn_error(p, abort, AERR_DRAIN);
+  } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax + epilogue
     // The four warps meet at named barriers, so none may leave the loop early:
     // after a failed wait a warp keeps going through every barrier with ok =
@@ -412,9 +426,13 @@ __global__ void __launch_bounds__(A_THREADS, 1)
 si_status launch_sparse_attention(const void* q, const void* kv, const int32_t* idx, int B, int S, int T, int k,
                                   float scale, void* out, float* lse, int* err, uint64_t wait_limit_ns,
                                   cudaStream_t stream) {
-  CUtensorMap tm_q;
+  CUtensorMap tm_q, tm_kv;
   si_status st = encode_tmap_2d(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, A_DK,
                                 static_cast<uint64_t>(B) * S * A_H, A_DK * 2, 64, A_H);
+  if (st != SI_OK) return st;
+  // the latents as [B*T rows, 576]: gather4 takes a box one row high
+  st = encode_tmap_2d(&tm_kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kv, A_DK, static_cast<uint64_t>(B) * T, A_DK * 2, 64,
+                      1);
   if (st != SI_OK) return st;
   int dev = 0, n_sm = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -437,7 +455,7 @@ si_status launch_sparse_attention(const void* q, const void* kv, const int32_t* 
   p.wait_limit_ns = wait_limit_ns;
   const long long nq = static_cast<long long>(B) * S;
   const int grid = static_cast<int>(std::min<long long>(nq, n_sm));
-  sparse_attn_kernel<<<grid, A_THREADS, smem, stream>>>(tm_q, p);
+  sparse_attn_kernel<<<grid, A_THREADS, smem, stream>>>(tm_q, tm_kv, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "sparse_attn_kernel launch");
   return SI_OK;

@@ -26,7 +26,7 @@
 namespace si {
 namespace {
 
-constexpr int kDefaultHostChunk = 8192;
+constexpr int kDefaultHostChunk = 4096;
 constexpr int kSlots = 2;
 
 struct HostPlan {

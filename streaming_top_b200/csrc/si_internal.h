@@ -62,7 +62,7 @@ si_status launch_merge_splits(const int32_t* part_idx, const float* part_score, 
                               int32_t* out_idx, float* out_score, cudaStream_t stream);
 // Key partitions per unit (1 = no split) and an upper bound of the partials'
 // bytes for a streaming call.
-int stream_split_count(long long n_units, int max_kt, int n_sm);
+int stream_split_count(long long n_units, int max_kt, int n_sm, int k);
 size_t stream_split_bytes_bound(int B, int S, int k, int query_chunk, int n_sm);
 
 // The streaming top-k over rows row0 .. row0+S-1 of every sequence (q, w

@@ -179,6 +179,7 @@ __global__ void __launch_bounds__(M_THREADS) merge_splits_kernel(const int32_t* 
     for (int sp = warp; sp < n_split; sp += M_WARPS) {
       uint64_t mn = ~0ull;
       uint32_t real = 0;
+#pragma unroll 4
       for (int i = lane; i < k; i += 32) {
         const uint64_t x = pack_entry(ps[sp * k + i], pi[sp * k + i]);
         if (x) {
@@ -201,6 +202,7 @@ __global__ void __launch_bounds__(M_THREADS) merge_splits_kernel(const int32_t* 
     const uint32_t take = total < static_cast<uint32_t>(k) ? total : static_cast<uint32_t>(k);
     const uint64_t bound = s_bound;
     // 2. the keys >= L into shared memory, while they fit
+#pragma unroll 4
     for (int i = tid; i < n; i += M_THREADS) {
       const uint64_t x = pack_entry(ps[i], pi[i]);
       if (x && x >= bound) {

@@ -451,6 +451,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       __syncwarp();
       const int t = U.t0 + q;
       int in_part = 0;
+      // the running state in registers between refreshes (st holds it for them)
+      uint32_t rn = 0, rbase = 0, rshift = 0;
+      bool rbinned = false;
       for (int j = U.kt0; j < U.kt1; ++j, ++tix) {
         const uint32_t slot = tix & (RING - 1), par = (tix / RING) & 1u;
         if (ok && !*abort && !mbar_wait_bounded(&C->ring_full[slot], par, abort, p.wait_limit_ns)) {
@@ -461,11 +464,18 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint64_t* area = ring + (slot * QT + q) * 4 * 32;
         if (ok && p.key_tile < KT) {
           // 64-key partitions: quadrants 0-1 hold keys 0-63 of the tile, 2-3 the rest
-          topk::merge(st, pool, area, C->ring_cnt[slot][q], 32, qh, lane, 0, 2);
+          topk::merge_r(rn, rbinned, rbase, rshift, pool, area, C->ring_cnt[slot][q], qh, lane, 0, 2);
+          __syncwarp();
+          if (lane == 0) st->cnt = rn;
+          __syncwarp();
           topk::refresh(st, pool, qh, k, p.cap, room, lane);
-          topk::merge(st, pool, area, C->ring_cnt[slot][q], 32, qh, lane, 2, 4);
+          {
+            const uint4 sv = *reinterpret_cast<const uint4*>(st);
+            rn = sv.x; rbase = sv.z; rshift = sv.w; rbinned = st->binned != 0;
+          }
+          topk::merge_r(rn, rbinned, rbase, rshift, pool, area, C->ring_cnt[slot][q], qh, lane, 2, 4);
         } else if (ok) {
-          topk::merge(st, pool, area, C->ring_cnt[slot][q], 32, qh, lane);
+          topk::merge_r(rn, rbinned, rbase, rshift, pool, area, C->ring_cnt[slot][q], qh, lane);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&C->ring_free[slot]);  // the slot has been read
@@ -474,8 +484,15 @@ __global__ void __launch_bounds__(THREADS, 1)
           in_part = 0;
           // at the unit's end only a histogram that does not exist yet is worth
           // building (finalize selects from it); no threshold is needed any more
-          if (ok && (!last || !st->binned)) {
+          __syncwarp();
+          if (lane == 0) st->cnt = rn;
+          __syncwarp();
+          if (ok && (!last || !rbinned)) {
             topk::refresh(st, pool, qh, k, p.cap, room, lane);
+            {
+              const uint4 sv = *reinterpret_cast<const uint4*>(st);
+              rn = sv.x; rbase = sv.z; rshift = sv.w; rbinned = st->binned != 0;
+            }
             if (lane == 0)
               *reinterpret_cast<volatile uint64_t*>(&C->pub[q]) = (static_cast<uint64_t>(i) << 32) | st->thr;
           }
@@ -650,12 +667,14 @@ bool stream_smem_plan(int k, int key_tile, int fp8, int* n_stages, int* pool_cap
 
 // Key partitions per unit for a launch of n_units units whose longest unit
 // spans max_kt key tiles: when the units cannot give every SM one, each
-// unit's keys are split over several CTAs (at least 4 tiles a partition).
-int stream_split_count(long long n_units, int max_kt, int n_sm) {
+// unit's keys are split over several CTAs (at least 4 tiles a partition, and
+// at most 32768 partial entries a row, which the merge selects from quickly).
+int stream_split_count(long long n_units, int max_kt, int n_sm, int k) {
   if (n_units <= 0 || n_units >= n_sm) return 1;
   const long long by_sm = n_sm / n_units;
   const long long by_len = max_kt / 4;
-  const long long s = std::min(by_sm, by_len);
+  const long long by_k = 32768 / k;
+  const long long s = std::min(std::min(by_sm, by_len), by_k);
   return s > 1 ? static_cast<int>(s) : 1;
 }
 
@@ -736,7 +755,7 @@ si_status launch_stream_topk(const void* q, const void* kc, const float* w, int 
     const int t_last = std::min(qt1 * QT, S) - 1;
     const long long n = std::min<long long>((static_cast<long long>(cfg.row0) + t_last + 1) / m, T);
     const int max_kt = static_cast<int>((n + KT - 1) / KT);
-    return cfg.allow_split ? stream_split_count(static_cast<long long>(B) * (qt1 - qt0), max_kt, n_sm) : 1;
+    return cfg.allow_split ? stream_split_count(static_cast<long long>(B) * (qt1 - qt0), max_kt, n_sm, k) : 1;
   };
   size_t part_bytes = 0;
   for (int qt0 = 0; qt0 < n_qt_total; qt0 += chunk_qt) {

@@ -362,49 +362,31 @@ __device__ __forceinline__ void pool_sort(uint64_t* pool, int n, int lane) {
   }
 }
 
-// merge(): move the query's candidates -- segments w_lo .. w_hi-1 of four,
-// segment w at area + w * seg_cap holding seg[w] entries -- to the end of its
-// main region in one pass over all lanes, counting them into the histogram
-// once it exists.  One warp.
-__device__ __forceinline__ void merge(QState* st, uint64_t* pool, const uint64_t* area,
-                                      const uint32_t* seg, int seg_cap, uint32_t* hist, int lane,
-                                      int w_lo = 0, int w_hi = 4) {
-  // every lane reads the four counts and the state with broadcast 16-byte loads
+// merge_r(): move the query's candidates -- segments w_lo .. w_hi-1 of four
+// 32-entry segments at `area`, segment w holding seg[w] entries -- to the end
+// of its main region, counting them into the histogram once it exists.  The
+// manager keeps its running state in registers between refreshes: n (the
+// main region's count) is updated in place, and binned / base / shift are
+// its copies of the histogram parameters.  One warp; the four segments'
+// loads are in flight together.
+__device__ __forceinline__ void merge_r(uint32_t& n, bool binned, uint32_t base, uint32_t shift, uint64_t* pool,
+                                        const uint64_t* area, const uint32_t* seg, uint32_t* hist, int lane,
+                                        int w_lo = 0, int w_hi = 4) {
   const uint4 cv = *reinterpret_cast<const uint4*>(seg);
-  const uint4 sv = *reinterpret_cast<const uint4*>(st);  // cnt, thr, base, shift
   const uint32_t c0 = w_lo <= 0 && 0 < w_hi ? cv.x : 0u, c1 = w_lo <= 1 && 1 < w_hi ? cv.y : 0u;
   const uint32_t c2 = w_lo <= 2 && 2 < w_hi ? cv.z : 0u, c3 = w_lo <= 3 && 3 < w_hi ? cv.w : 0u;
-  const uint32_t o1 = c0, o2 = c0 + c1, o3 = c0 + c1 + c2, tot = o3 + c3;
-  const uint32_t n = sv.x;
-  const bool binned = st->binned != 0;
-  const uint32_t base = sv.z, shift = sv.w;
-  if (seg_cap == 32) {
-    // one independent copy per segment: the four loads are in flight together
-    const uint32_t cw[4] = {c0, c1, c2, c3}, ow[4] = {0u, o1, o2, o3};
-    uint64_t x[4];
+  const uint32_t cw[4] = {c0, c1, c2, c3}, ow[4] = {0u, c0, c0 + c1, c0 + c1 + c2};
+  uint64_t x[4];
 #pragma unroll
-    for (int w = 0; w < 4; ++w) x[w] = static_cast<uint32_t>(lane) < cw[w] ? area[w * 32 + lane] : 0ull;
+  for (int w = 0; w < 4; ++w) x[w] = static_cast<uint32_t>(lane) < cw[w] ? area[w * 32 + lane] : 0ull;
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      if (static_cast<uint32_t>(lane) < cw[w]) {
-        pool[n + ow[w] + lane] = x[w];
-        if (binned) atomicAdd(&hist[bin_of(static_cast<uint32_t>(x[w] >> 32), base, shift)], 1u);
-      }
-    }
-  } else {
-    for (uint32_t r = lane; r < tot; r += 32) {
-      // segment w holds ranks [o_w, o_w + c_w)
-      const uint32_t src = r >= o3 ? 3u * seg_cap + (r - o3)
-                           : r >= o2 ? 2u * seg_cap + (r - o2)
-                           : r >= o1 ? 1u * seg_cap + (r - o1) : r;
-      const uint64_t x = area[src];
-      pool[n + r] = x;
-      if (binned) atomicAdd(&hist[bin_of(static_cast<uint32_t>(x >> 32), base, shift)], 1u);
+  for (int w = 0; w < 4; ++w) {
+    if (static_cast<uint32_t>(lane) < cw[w]) {
+      pool[n + ow[w] + lane] = x[w];
+      if (binned) atomicAdd(&hist[bin_of(static_cast<uint32_t>(x[w] >> 32), base, shift)], 1u);
     }
   }
-  __syncwarp();
-  if (lane == 0) st->cnt = n + tot;
-  __syncwarp();
+  n += c0 + c1 + c2 + c3;
 }
 
 // refresh(), at the end of a partition of keys:
