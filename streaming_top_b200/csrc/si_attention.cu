@@ -24,9 +24,8 @@
 //        per stage), B = P^T; fp32 into TMEM columns [256 + 64 v, ...) for dv
 //        tile v.
 //   out  O[t, h, dv] = O^T * (1 / sum_h), bf16; lse[t, h] fp32.
-// Warps: 0 q loads (TMA), 1 MMA issue, 2 gather producer (TMA gather4: four
-// latent rows a lane, a 16 KB stage a warp instruction), 3 idle, 4-7 softmax
-// and epilogue.  Every wait
+// Warps: 0 q loads (TMA), 1 MMA issue, 2-3 gather producers (half of each
+// stage by TMA gather4, half by 16-byte cp.async), 4-7 softmax and epilogue.  Every wait
 // is bounded; on expiry the kernel records SI_ERR_TIMEOUT, drains its copies
 // and MMAs and exits.
 #include <cuda.h>
@@ -66,13 +65,26 @@ struct AttnParams {
 
 struct ACtrl {
   uint64_t full[A_NS], empty[A_NS];
-  uint64_t q_full, q_empty, s_full, p_full, o_full, o_empty, done;
+  uint64_t q_full, q_empty, s_full, o_full, o_empty, done;
+  uint64_t p_full[4];     // per 128-entry tile: its rounded weights are in P^T
   uint32_t tmem_slot;
   int abort;
   float red[4][A_H];      // per-quadrant partial max / sum
-  float head_max[A_H], head_inv[A_H];  // per head: max logit, 1 / sum of the rounded weights
-  alignas(16) int sel[A_KMAX];  // the producer's copy of the current query's selection: latent rows
+  alignas(16) float head_max[A_H];  // per head: max logit (read as float4)
+  float head_inv[A_H];              // per head: 1 / sum of the rounded weights
+  alignas(16) int sel[2][A_KMAX];  // each producer warp's copy of the current query's selection: latent rows
 };
+
+// 16-byte global -> shared copy (L2 only).
+__device__ __forceinline__ void cp16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+// The barrier receives one arrival when every cp.async this thread has issued
+// so far has landed (its expected count includes that arrival).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
 
 // TMA gather of four rows r0..r3 of a 2-D tensor map (box: 64 elements x 1
 // row), columns x .. x+63, into four consecutive 128-byte rows at dst
@@ -122,13 +134,13 @@ __global__ void __launch_bounds__(A_THREADS, 1)
   const int qk_stages = n_et * A_KB, pv_stages = 4 * n_kc;
   if (threadIdx.x == 0) {
     for (int s = 0; s < A_NS; ++s) {
-      mbar_init(&C->full[s], 1);
+      mbar_init(&C->full[s], 33);  // warp 2's expect-tx arrival + one noinc arrival per lane of warp 3
       mbar_init(&C->empty[s], 1);
     }
     mbar_init(&C->q_full, 1);
     mbar_init(&C->q_empty, 1);
     mbar_init(&C->s_full, 1);
-    mbar_init(&C->p_full, 128);
+    for (int j = 0; j < 4; ++j) mbar_init(&C->p_full[j], 128);
     mbar_init(&C->o_full, 1);
     mbar_init(&C->o_empty, 128);
     mbar_init(&C->done, 1);
@@ -184,6 +196,7 @@ __global__ void __launch_bounds__(A_THREADS, 1)
               break;
             }
             tc_fence_after();
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // cp.async data -> MMA operand
             const uint32_t a0 = sa + stage * A_STAGE;
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
@@ -198,23 +211,27 @@ __global__ void __launch_bounds__(A_THREADS, 1)
         if (stop) break;
         mma_commit(&C->s_full);
         mma_commit(&C->q_empty);
-        if (!mbar_wait_bounded(&C->p_full, par, abort, p.wait_limit_ns)) {
-          attn_error(p, abort, AERR_P_FULL);
-          break;
-        }
         if (!mbar_wait_bounded(&C->o_empty, par ^ 1u, abort, p.wait_limit_ns)) {
           attn_error(p, abort, AERR_O_FREE);
           break;
         }
-        tc_fence_after();
-        for (int vt = 0; vt < 4 && !stop; ++vt)
-          for (int c = 0; c < n_kc; ++c) {
+        // PV chunk by chunk (64 entries, the four dv tiles each): a tile's two
+        // chunks start as soon as the softmax warps have written its weights
+        for (int c = 0; c < n_kc && !stop; ++c) {
+          if ((c & 1) == 0 && !mbar_wait_bounded(&C->p_full[c >> 1], par, abort, p.wait_limit_ns)) {
+            attn_error(p, abort, AERR_P_FULL);
+            stop = true;
+            break;
+          }
+          tc_fence_after();
+          for (int vt = 0; vt < 4; ++vt) {
             if (!mbar_wait_bounded(&C->full[stage], phase, abort, p.wait_limit_ns)) {
               attn_error(p, abort, AERR_STAGE_FULL);
               stop = true;
               break;
             }
             tc_fence_after();
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // cp.async data -> MMA operand
             const uint32_t a0 = sa + stage * A_STAGE;
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)  // 16 entries a step: two 8-entry atom rows
@@ -226,69 +243,103 @@ __global__ void __launch_bounds__(A_THREADS, 1)
               phase ^= 1u;
             }
           }
+        }
         if (!stop) mma_commit(&C->o_full);
       }
       // every MMA issued above has completed before TMEM is released
       mma_commit(&C->done);
       if (!mbar_wait_timed(&C->done, 0, p.wait_limit_ns)) attn_error(p, abort, AERR_DRAIN);
     }
-  } else if (warp == 2) {
-    // ------------------------------------------------------------ gather producer (TMA gather4)
-    // The warp copies the query's selection into shared memory, then fills
-    // each 16 KB stage with one gather4 per lane: 4 latent rows x 64 dims
-    // (512 B) each, landing in the 128-byte-swizzled layout the MMA reads.
-    // One warp instruction issues the whole stage; lane 0 owns the barriers.
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ gather producers
+    // Two copy paths fill each 16 KB stage side by side: warp 2 through the
+    // TMA unit (one gather4 of 4 latent rows x 128 B per lane, 16 lanes: half
+    // the stage), warp 3 through the load/store path (16-byte cp.async, eight
+    // lanes to a row: the other half).  The rows land in the 128-byte-swizzled
+    // layout the MMA reads.  Each warp keeps its own copy of the selection, so
+    // the two never wait for each other.  The stage's barrier takes warp 2's
+    // expect-tx arrival and one noinc arrival per lane of warp 3.
+    const bool tma = warp == 2;
+    int* sel = C->sel[warp - 2];
     uint32_t stage = 0, phase = 0;
-    uint32_t any_load = 0, last_par = 0;  // per stage: loaded at all / parity of the last load
+    uint32_t any_load = 0, last_par = 0;  // warp 2, per stage: loaded at all / parity of the last load
     bool stop = false;
+    // the selection of the warp's next query, loaded while the current one's
+    // stages are issued
+    int nxt[A_KMAX / 32];
+#pragma unroll
+    for (int i = 0; i < A_KMAX / 32; ++i)
+      nxt[i] = q0 < nq && 32 * i < p.k ? p.idx[static_cast<size_t>(q0) * p.k + 32 * i + lane] : 0;
     for (int t = q0; t < nq && !stop; t += qstep) {
-      const int row_base = (t / p.S) * p.T;  // the sequence's first latent row in the tensor map
-      __syncwarp();  // every lane has issued its loads of the last query
-      for (int e = lane; e < p.k; e += 32) {
-        const int key = p.idx[static_cast<size_t>(t) * p.k + e];
-        C->sel[e] = row_base + (key >= 0 && key < p.T ? key : 0);  // padding reads row 0; its weight is 0
-      }
+      const int row_base = (t / p.S) * p.T;  // the sequence's first latent row
+      __syncwarp();                          // the warp's copies of the last query have read sel
+#pragma unroll
+      for (int i = 0; i < A_KMAX / 32; ++i)
+        if (32 * i < p.k) {
+          const int key = nxt[i];
+          sel[32 * i + lane] = row_base + (key >= 0 && key < p.T ? key : 0);  // padding reads row 0; weight 0
+        }
       __syncwarp();
+      const int tn = t + qstep;
+#pragma unroll
+      for (int i = 0; i < A_KMAX / 32; ++i)
+        nxt[i] = tn < nq && 32 * i < p.k ? p.idx[static_cast<size_t>(tn) * p.k + 32 * i + lane] : 0;
       for (int j = 0; j < qk_stages + pv_stages; ++j) {
         bool got = true;
         if (lane == 0) {
           got = mbar_wait_bounded(&C->empty[stage], phase ^ 1u, abort, p.wait_limit_ns);
-          if (got)
-            mbar_arrive_expect_tx(&C->full[stage], A_STAGE);
-          else
+          if (!got)
             attn_error(p, abort, AERR_STAGE_FREE);
+          else if (tma)
+            mbar_arrive_expect_tx(&C->full[stage], A_STAGE / 2);
         }
         if (__shfl_sync(0xFFFFFFFFu, got ? 1 : 0, 0) == 0) {
           stop = true;
           break;
         }
         __syncwarp();
-        int e, x, off;
-        if (j < qk_stages) {  // entry tile j / 9, K-block j % 9: 128 rows x 128 B
-          e = (j / A_KB) * 128 + 4 * lane;
-          x = (j % A_KB) * 64;
-          off = lane * 512;
-        } else {  // dv tile, 64-entry chunk: two atoms (64 dv each) of 64 rows x 128 B
-          const int jj = j - qk_stages, a = lane >> 4;
-          e = (jj % n_kc) * 64 + 4 * (lane & 15);
-          x = (jj / n_kc) * 128 + a * 64;
-          off = a * 8192 + (lane & 15) * 512;
+        uint8_t* dst = st_s + stage * A_STAGE;
+        // QK stage (entry tile j / 9, K-block j % 9): 128 rows x 128 B; TMA rows
+        // 0-63, cp.async rows 64-127.  PV stage (64-entry chunk jj / 4, dv tile
+        // jj % 4): two atoms (64 dv each) of 64 rows x 128 B; TMA atom 0,
+        // cp.async atom 1.
+        const bool qk = j < qk_stages;
+        const int jj = j - qk_stages;
+        const int e0 = qk ? (j / A_KB) * 128 : (jj >> 2) * 64;
+        const int x = qk ? (j % A_KB) * 64 : (jj & 3) * 128;
+        if (tma) {
+          if (lane < 16) {
+            const int4 r = *reinterpret_cast<const int4*>(&sel[e0 + 4 * lane]);
+            tma_gather4(dst + lane * 512, &tm_kv, &C->full[stage], x, r.x, r.y, r.z, r.w);
+          }
+          any_load |= 1u << stage;
+          last_par = (last_par & ~(1u << stage)) | (phase << stage);
+        } else {
+          const uint32_t base = smem_u32(dst) + 8192u;  // rows 64-127 of a QK stage, atom 1 of a PV stage
+          const int ro = qk ? 64 : 0, xo = qk ? x : x + 64;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int id = lane + 32 * i, row = id >> 3, ch = id & 7;
+            cp16(base + row * 128 + ((ch ^ (row & 7)) << 4),
+                 p.kv + static_cast<size_t>(sel[e0 + ro + row]) * (A_DK * 2) + xo * 2 + ch * 16);
+          }
+          cp_async_arrive_noinc(&C->full[stage]);
         }
-        const int4 r = *reinterpret_cast<const int4*>(&C->sel[e]);
-        tma_gather4(st_s + stage * A_STAGE + off, &tm_kv, &C->full[stage], x, r.x, r.y, r.z, r.w);
-        any_load |= 1u << stage;
-        last_par = (last_par & ~(1u << stage)) | (phase << stage);
         if (++stage == A_NS) {
           stage = 0;
           phase ^= 1u;
         }
       }
     }
-    // every load issued has landed before the CTA can exit
-    if (lane == 0)
-      for (int s = 0; s < A_NS; ++s)
-        if (((any_load >> s) & 1u) && !mbar_wait_timed(&C->full[s], (last_par >> s) & 1u, p.wait_limit_ns))
-          attn_error(p, abort, AERR_DRAIN);
+    // every copy issued has landed before the CTA can exit
+    if (tma) {
+      if (lane == 0)
+        for (int s = 0; s < A_NS; ++s)
+          if (((any_load >> s) & 1u) && !mbar_wait_timed(&C->full[s], (last_par >> s) & 1u, p.wait_limit_ns))
+            attn_error(p, abort, AERR_DRAIN);
+    } else {
+      asm volatile("cp.async.wait_all;" ::: "memory");
+    }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax + epilogue
     // The four warps meet at named barriers, so none may leave the loop early:
@@ -300,12 +351,12 @@ __global__ void __launch_bounds__(A_THREADS, 1)
     bool ok = true;
     for (int t = q0; t < nq; t += qstep, ++n) {
       const uint32_t par = n & 1u;
-      bool valid[4];
+      uint32_t vmask = 0;  // bit jt: this thread's entry of tile jt is a real key
 #pragma unroll
       for (int jt = 0; jt < 4; ++jt) {
-        const int e = jt * 128 + quad * 32 + lane;
-        valid[jt] = jt < n_et && p.idx[static_cast<size_t>(t) * p.k + e] >= 0 &&
-                    p.idx[static_cast<size_t>(t) * p.k + e] < p.T;
+        if (jt >= n_et) break;
+        const int key = p.idx[static_cast<size_t>(t) * p.k + jt * 128 + quad * 32 + lane];
+        vmask |= (key >= 0 && key < p.T ? 1u : 0u) << jt;
       }
       const bool got = ok && mbar_wait_bounded(&C->s_full, par, abort, p.wait_limit_ns);
       if (ok && !__all_sync(0xFFFFFFFFu, got)) {
@@ -313,18 +364,18 @@ __global__ void __launch_bounds__(A_THREADS, 1)
         ok = false;
       }
       tc_fence_after();
-      // two passes of 32 heads keep the live arrays at 3 x 32 registers
+      // 1. per-head maximum over the valid entries, in two halves of 32 heads
+#pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
-        float m[32], sum[32];
+        float m[32];
         uint32_t x[32];
 #pragma unroll
         for (int h = 0; h < 32; ++h) m[h] = ninf;
-#pragma unroll
-        for (int jt = 0; jt < 4; ++jt) {
-          if (jt >= n_et || !ok) break;
+#pragma unroll 1
+        for (int jt = 0; jt < n_et && ok; ++jt) {
           tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + jt * A_H + hh * 32, x);
           tmem_ld_wait();
-          if (valid[jt]) {
+          if ((vmask >> jt) & 1u) {
 #pragma unroll
             for (int h = 0; h < 32; ++h) m[h] = fmaxf(m[h], __uint_as_float(x[h]));
           }
@@ -333,66 +384,75 @@ __global__ void __launch_bounds__(A_THREADS, 1)
         for (int h = 0; h < 32; ++h)
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) m[h] = fmaxf(m[h], __shfl_xor_sync(0xFFFFFFFFu, m[h], o));
-        {
-          float mine = 0.f;  // m[lane] without a dynamic register index
+        float mine = 0.f;  // m[lane] without a dynamic register index
 #pragma unroll
-          for (int h = 0; h < 32; ++h) mine = h == lane ? m[h] : mine;
-          C->red[quad][hh * 32 + lane] = mine;
-        }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+        for (int h = 0; h < 32; ++h) mine = h == lane ? m[h] : mine;
+        C->red[quad][hh * 32 + lane] = mine;
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (quad == 0)
+        for (int hg = lane; hg < A_H; hg += 32)
+          C->head_max[hg] = fmaxf(fmaxf(C->red[0][hg], C->red[1][hg]), fmaxf(C->red[2][hg], C->red[3][hg]));
+      asm volatile("bar.sync 1, 128;" ::: "memory");  // head_max is complete; red is free
+      // 2. tile by tile, the rounded weights of all heads into P^T; each tile's
+      //    barrier lets the MMA warp start that tile's PV while the next is done
+      float sum[A_H];
 #pragma unroll
-        for (int h = 0; h < 32; ++h) {
-          const int hg = hh * 32 + h;
-          m[h] = fmaxf(fmaxf(C->red[0][hg], C->red[1][hg]), fmaxf(C->red[2][hg], C->red[3][hg]));
-        }
-        if (quad == 0) {
-          float mine = 0.f;
-#pragma unroll
-          for (int h = 0; h < 32; ++h) mine = h == lane ? m[h] : mine;
-          C->head_max[hh * 32 + lane] = mine;
-        }
-        asm volatile("bar.sync 1, 128;" ::: "memory");  // red is reused for the sums
-#pragma unroll
-        for (int h = 0; h < 32; ++h) sum[h] = 0.f;
-#pragma unroll
-        for (int jt = 0; jt < 4; ++jt) {
-          if (jt >= n_et || !ok) break;
-          tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + jt * A_H + hh * 32, x);
-          tmem_ld_wait();
+      for (int h = 0; h < A_H; ++h) sum[h] = 0.f;
+#pragma unroll 1
+      for (int jt = 0; jt < n_et; ++jt) {
+        if (ok) {
           const int e = jt * 128 + quad * 32 + lane, kb = e >> 6, col = e & 63;
+          const bool valid = (vmask >> jt) & 1u;
 #pragma unroll
-          for (int h = 0; h < 32; ++h) {
-            const int hg = hh * 32 + h;
-            const float pr = valid[jt] ? __expf(p.scale * (__uint_as_float(x[h]) - m[h])) : 0.f;
-            const __nv_bfloat16 pb = __float2bfloat16_rn(pr);
-            sum[h] += __bfloat162float(pb);
-            // P^T K-major: block kb = [64 heads][64 entries], row hg, swizzled 16-byte chunk
-            const int off = kb * 8192 + hg * 128 + ((((col * 2) >> 4) ^ (hg & 7)) << 4) + ((col * 2) & 15);
-            *reinterpret_cast<__nv_bfloat16*>(p_s + off) = pb;
+          for (int hh = 0; hh < 2; ++hh) {
+            uint32_t x[32];
+            tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + jt * A_H + hh * 32, x);
+            tmem_ld_wait();
+#pragma unroll
+            for (int h4 = 0; h4 < 32; h4 += 4) {
+              const float4 mx = *reinterpret_cast<const float4*>(&C->head_max[hh * 32 + h4]);
+              const float mv[4] = {mx.x, mx.y, mx.z, mx.w};
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const int h = h4 + u, hg = hh * 32 + h;
+                const float pr = valid ? __expf(p.scale * (__uint_as_float(x[h]) - mv[u])) : 0.f;
+                const __nv_bfloat16 pb = __float2bfloat16_rn(pr);
+                sum[hg] += __bfloat162float(pb);
+                // P^T K-major: block kb = [64 heads][64 entries], row hg, swizzled 16-byte chunk
+                const int off = kb * 8192 + hg * 128 + ((((col * 2) >> 4) ^ (hg & 7)) << 4) + ((col * 2) & 15);
+                *reinterpret_cast<__nv_bfloat16*>(p_s + off) = pb;
+              }
+            }
           }
         }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // P is read by the MMA (async proxy)
+        tc_fence_before();
+        mbar_arrive(&C->p_full[jt]);
+      }
+      // 3. per-head sums of the rounded weights -> 1 / sum and the log-sum-exp
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        float v[32];
+#pragma unroll
+        for (int h = 0; h < 32; ++h) v[h] = sum[hh * 32 + h];
 #pragma unroll
         for (int h = 0; h < 32; ++h)
 #pragma unroll
-          for (int o = 16; o > 0; o >>= 1) sum[h] += __shfl_xor_sync(0xFFFFFFFFu, sum[h], o);
-        {
-          float mine = 0.f;
+          for (int o = 16; o > 0; o >>= 1) v[h] += __shfl_xor_sync(0xFFFFFFFFu, v[h], o);
+        float mine = 0.f;
 #pragma unroll
-          for (int h = 0; h < 32; ++h) mine = h == lane ? sum[h] : mine;
-          C->red[quad][hh * 32 + lane] = mine;
-        }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (quad == 0) {
-          const int hg = hh * 32 + lane;
+        for (int h = 0; h < 32; ++h) mine = h == lane ? v[h] : mine;
+        C->red[quad][hh * 32 + lane] = mine;
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (quad == 0)
+        for (int hg = lane; hg < A_H; hg += 32) {
           const float s = C->red[0][hg] + C->red[1][hg] + C->red[2][hg] + C->red[3][hg];
           C->head_inv[hg] = s > 0.f ? 1.0f / s : 0.f;
           if (ok) p.lse[static_cast<size_t>(t) * A_H + hg] = s > 0.f ? p.scale * C->head_max[hg] + __logf(s) : ninf;
         }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-      }
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // P is read by the MMA (async proxy)
-      tc_fence_before();
-      mbar_arrive(&C->p_full);
+      asm volatile("bar.sync 1, 128;" ::: "memory");  // head_inv is complete
       // epilogue: lane = dv, 64 heads a load
       const bool gotO = ok && mbar_wait_bounded(&C->o_full, par, abort, p.wait_limit_ns);
       if (ok && !__all_sync(0xFFFFFFFFu, gotO)) {
