@@ -757,7 +757,8 @@ def run_attention(args, wl):
         "config": {"workload": f"sparse attention at the {wl.name} shape: B={wl.B}, S={wl.S} queries x 64 heads, "
                                f"T={wl.T} latents of 576 (values: the first 512), the indexer's top-{wl.k} "
                                f"of the planted inputs (seed {wl.seed}) as the selection",
-                   "selected_entries": sel, "l2": "q (4.8 GB) > L2, and L2 flushed before each timed step"},
+                   "selected_entries": sel,
+                   "l2": f"q ({qd.numel() * 2 / 1e9:.1f} GB) > L2, and L2 flushed before each timed step"},
         "tflops": flop / (ms * 1e-3) / 1e12,
         "roofline": {"bound": "tensor", "kernel": "sparse_attn_kernel", "achieved": flop / (ms * 1e-3) / 1e12,
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
