@@ -304,6 +304,42 @@ def test_row_sort_matches_lexicographic_order(k):
         assert np.array_equal(np.abs(gs[r]), np.abs(sc[r][order])), r
 
 
+@pytest.mark.parametrize("k", [257, 384, 512])
+@pytest.mark.parametrize("kind", ["gauss", "narrow", "early_rows"])
+def test_row_sort_distinct_and_clustered_scores(k, kind):
+    """si_sort_topk_rows on rows whose scores are mostly distinct (the shape
+    the streaming kernel hands over): Gaussian, a narrow cluster with a few
+    outliers and exact ties, and early-row shapes with a long padding tail.
+    Score descending, index ascending, (-1, -inf) padding last."""
+    rng = np.random.default_rng(1000 + k)
+    rows = 256
+    idx = rng.permutation(rows * k).astype(np.int32).reshape(rows, k)
+    if kind == "gauss":
+        sc = rng.standard_normal((rows, k)).astype(np.float32)
+    else:
+        sc = (5.0 + 1e-3 * rng.standard_normal((rows, k))).astype(np.float32)
+        sc[:, :3] = np.float32([40.0, -7.0, 5.0])
+    tie = rng.random((rows, k)) < 0.05
+    sc[tie] = sc[:, :1].repeat(k, axis=1)[tie]  # exact ties with the row's first score
+    if kind == "early_rows":
+        n_real = rng.integers(0, k + 1, size=rows)
+        pad = np.arange(k)[None, :] >= n_real[:, None]
+    else:
+        pad = rng.random((rows, k)) < 0.1
+    idx[pad] = -1
+    sc[pad] = -np.inf
+    ti, ts = torch.from_numpy(idx).cuda(), torch.from_numpy(sc).cuda()
+    si.sort_topk_rows(ti, ts)
+    assert si.device_status() == si.SI_OK
+    gi, gs = ti.cpu().numpy(), ts.cpu().numpy()
+    for r in range(rows):
+        s = np.where(idx[r] < 0, -np.inf, sc[r]).astype(np.float64) + 0.0
+        key_idx = np.where(idx[r] < 0, np.iinfo(np.int64).max, idx[r].astype(np.int64))
+        order = np.lexsort((key_idx, -s))
+        assert np.array_equal(gi[r], idx[r][order]), r
+        assert np.array_equal(gs[r], sc[r][order]), r
+
+
 def test_default_key_tile_falls_back_for_large_k():
     """k=2048 with the default partition: the library picks a partition whose
     pool fits (an explicit 512 is refused) and the result is exact."""
