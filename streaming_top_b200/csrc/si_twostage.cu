@@ -87,6 +87,7 @@ struct FineParams {
   int nb;                  // complete blocks of the sequence, T / G
   int g_shift;             // log2(G) when G is a power of two, else -1 (divide)
   long long row0;          // absolute position of chunk row 0
+  int box_rows;            // 4 or 8: candidates arrive by TMA boxes of that many key rows; 0: cp.async
   uint64_t wait_limit_ns;
 };
 
@@ -199,7 +200,8 @@ __device__ __forceinline__ FUnit f_decode(const FineParams& p, int u, int n_unit
 }
 
 __global__ void __launch_bounds__(F_THREADS, 1)
-    fine_score_kernel(const __grid_constant__ CUtensorMap tm_q, const FineParams p) {
+    fine_score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kc,
+                      const FineParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -212,7 +214,7 @@ __global__ void __launch_bounds__(F_THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < F_STAGES; ++s) {
-      mbar_init(&C->full[s], F_PRODUCERS);
+      mbar_init(&C->full[s], p.box_rows ? 1 : F_PRODUCERS);
       mbar_init(&C->empty[s], 1);
     }
     mbar_init(&C->q_full, 1);
@@ -225,7 +227,10 @@ __global__ void __launch_bounds__(F_THREADS, 1)
     *abort = 0;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) prefetch_tmap(&tm_q);
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tm_q);
+    if (p.box_rows) prefetch_tmap(&tm_kc);
+  }
   if (warp == 1) tmem_alloc(&C->tmem_slot, 256);
   tc_fence_before();
   __syncthreads();
@@ -314,6 +319,74 @@ __global__ void __launch_bounds__(F_THREADS, 1)
       }
       mma_commit(&C->mma_done);
       if (!mbar_wait_timed(&C->mma_done, 0, p.wait_limit_ns)) f_record(p, abort, FERR_DRAIN);
+    }
+  } else if (warp < 4 && p.box_rows) {
+    // ------------------------------------------------------------ gather producer (TMA boxes)
+    // Every group of 8 candidate slots is 8 consecutive key rows that start
+    // on a multiple of gcd(G, 8): a kept block's keys (or 8 of them) or the
+    // incomplete block's.  Warp 2, lane l, loads group l % 16 of query l / 16
+    // as 8 / box_rows TMA boxes of box_rows rows x 64 dims per K half (one
+    // 1 KB, 128-byte-swizzled atom of the stage); lane 0 owns the barriers.
+    // Slots past the row's candidates read key row 0 (their scores are never
+    // stored), rows past the keys read as zero.  Warp 3 has nothing to do.
+    if (warp == 2) {
+      const bool j1 = (lane >> 4) != 0;  // this lane's query, chosen without a dynamic index
+      const int bb = lane & 15, nsub = 8 / p.box_rows;
+      uint32_t stage = 0, phase = 0;
+      uint32_t any_load = 0, last_par = 0;  // per stage: loaded at all / parity of the last load
+      bool stop = false;
+      for (int i = 0; !stop; ++i) {
+        const int u = f_unit_of(i, n_units);
+        if (u < 0 || __any_sync(0xFFFFFFFFu, *abort != 0)) break;  // the warp decides as one
+        const FUnit U = f_decode(p, u, n_units);
+        const int rj = j1 ? U.r[1] : U.r[0];
+        const Cand c = j1 ? U.c[1] : U.c[0];
+        const int32_t* crow = p.coarse + static_cast<size_t>(rj < p.R ? rj : 0) * p.n_keep;
+        for (int t = 0; t < U.nt && !stop; ++t) {
+          int row[2];
+#pragma unroll
+          for (int x = 0; x < 2; ++x) {
+            const int s1 = t * F_KT + 8 * bb + x * 4;
+            int kr = 0;
+            if (s1 < c.n_blk_keys) {
+              const int blk = crow[min(blk_slot(p, s1), p.n_keep - 1)];
+              kr = blk >= 0 && blk < p.nb ? blk * p.G + in_blk(p, s1) : 0;
+            } else if (s1 < c.count) {
+              kr = c.tail0 + (s1 - c.n_blk_keys);
+            }
+            row[x] = kr;
+          }
+          for (int h = 0; h < 2; ++h) {
+            bool got = true;
+            if (lane == 0) {
+              got = mbar_wait_bounded(&C->empty[stage], phase ^ 1u, abort, p.wait_limit_ns);
+              if (!got)
+                f_record(p, abort, FERR_EMPTY);
+              else
+                mbar_arrive_expect_tx(&C->full[stage], F_STAGE_BYTES);
+            }
+            if (__shfl_sync(0xFFFFFFFFu, got ? 1 : 0, 0) == 0) {  // the warp gives up as one
+              stop = true;
+              break;
+            }
+            __syncwarp();
+            uint8_t* dst = a_s + stage * F_STAGE_BYTES + (j1 ? F_A_QUERY : 0) + bb * 1024;
+            tma_load_2d(dst, &tm_kc, &C->full[stage], h * 64, row[0]);
+            if (nsub == 2) tma_load_2d(dst + 512, &tm_kc, &C->full[stage], h * 64, row[1]);
+            any_load |= 1u << stage;
+            last_par = (last_par & ~(1u << stage)) | (phase << stage);
+            if (++stage == F_STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+        }
+      }
+      // every load issued has landed before the CTA can exit
+      if (lane == 0)
+        for (int s2 = 0; s2 < F_STAGES; ++s2)
+          if (((any_load >> s2) & 1u) && !mbar_wait_timed(&C->full[s2], (last_par >> s2) & 1u, p.wait_limit_ns))
+            f_record(p, abort, FERR_DRAIN);
     }
   } else if (warp < 4) {
     // ------------------------------------------------------------ gather producers
@@ -661,10 +734,20 @@ si_status launch_two_stage(const void* q, const void* kc, const float* w, int B,
                                 n_keep, coarse, nullptr, stream, cfg);
         if (st != SI_OK) break;
       }
-      CUtensorMap tm_q;
+      CUtensorMap tm_q, tm_kc;
       st = encode_tmap_2d(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, qb, F_DIM, static_cast<uint64_t>(R) * F_HEADS,
                           F_DIM * 2, 64, F_QT * F_HEADS);
       if (st != SI_OK) break;
+      // candidates come in runs of gcd(G, 8) consecutive key rows starting on
+      // a multiple of it; runs of 4 or 8 rows load as TMA boxes of the keys
+      const int box_rows = (G % 8 == 0) ? 8 : (G % 4 == 0) ? 4 : 0;
+      tm_kc = tm_q;  // unused unless box_rows
+      if (box_rows) {
+        st = encode_tmap_2d(&tm_kc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                            static_cast<const uint8_t*>(kc) + static_cast<size_t>(b) * T * F_DIM * 2, F_DIM,
+                            static_cast<uint64_t>(T), F_DIM * 2, 64, box_rows);
+        if (st != SI_OK) break;
+      }
       FineParams fp;
       fp.kc = static_cast<const uint8_t*>(kc) + static_cast<size_t>(b) * T * F_DIM * 2;
       fp.w = wb;
@@ -680,9 +763,10 @@ si_status launch_two_stage(const void* q, const void* kc, const float* w, int B,
       fp.nb = nb;
       fp.g_shift = (G & (G - 1)) == 0 ? __builtin_ctz(static_cast<unsigned>(G)) : -1;
       fp.row0 = c0;
+      fp.box_rows = box_rows;
       fp.wait_limit_ns = wait_limit_ns;
       const int units = (R + F_QT - 1) / F_QT;
-      fine_score_kernel<<<static_cast<unsigned>(std::min(units, n_sm)), F_THREADS, F_SMEM, stream>>>(tm_q, fp);
+      fine_score_kernel<<<static_cast<unsigned>(std::min(units, n_sm)), F_THREADS, F_SMEM, stream>>>(tm_q, tm_kc, fp);
       e = cudaGetLastError();
       if (e != cudaSuccess) {
         st = cuda_fail(e, "fine_score_kernel launch");
