@@ -38,6 +38,11 @@ si_status scratch_alloc(void** p, size_t bytes, cudaStream_t stream, const char*
 si_status encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
                          uint64_t inner, uint64_t outer, uint64_t row_bytes, uint32_t box_inner,
                          uint32_t box_outer);
+// 3-D tiled tensor map (128-byte swizzle): dims[0] contiguous, strides (in
+// bytes) of dims 1 and 2 in any order.  Returns false, recording no error,
+// when the driver refuses the layout (the caller then uses 2-D boxes).
+bool try_encode_tmap_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, const uint64_t dims[3],
+                        const uint64_t stride_bytes[2], const uint32_t box[3]);
 
 struct StreamConfig {
   int query_chunk;  // queries per launch (multiple of 4), or S

@@ -44,13 +44,17 @@ constexpr int F_HEADS = 64;
 constexpr int F_DIM = 128;
 constexpr int F_KT = 128;                // candidates per tile (MMA M)
 constexpr int F_THREADS = 384;           // 12 warps
-constexpr int F_STAGES = 6;              // K-half stages of shared memory
-constexpr int F_IN_FLIGHT = 4;           // copy groups a producer thread keeps outstanding
-constexpr int F_PRODUCERS = 64;          // warps 2, 3 fill every stage together
+constexpr int F_STAGES = 3;              // candidate-tile stages of shared memory
+constexpr int F_PRODUCERS = 64;          // cp.async path: warps 2, 3 fill every stage together
 constexpr int F_Q_HALF = F_QT * F_HEADS * 128;        // 16 KB: one 64-column half of the q tile
 constexpr int F_Q_BYTES = 2 * F_Q_HALF;               // 32 KB
-constexpr int F_A_QUERY = F_KT * 128;                 // 16 KB: one query's keys, one K half
-constexpr int F_STAGE_BYTES = F_QT * F_A_QUERY;       // 32 KB
+// A stage holds one candidate tile of both queries, both K halves: query j's
+// 128 rows in 16 groups of 8 (2 KB each), a group's half h at +1 KB, each a
+// 1 KB 128-byte-swizzled atom of 8 rows x 64 dims.  The MMA reads a half as
+// K-major rows with 2 KB between 8-row groups.
+constexpr int F_GROUP = 2048;                         // 8 rows x 2 halves x 128 B
+constexpr int F_A_QUERY = F_KT / 8 * F_GROUP;         // 32 KB: one query's tile
+constexpr int F_STAGE_BYTES = F_QT * F_A_QUERY;       // 64 KB
 constexpr int F_CTRL_BYTES = 256;
 constexpr int F_SMEM = F_Q_BYTES + F_STAGES * F_STAGE_BYTES + F_CTRL_BYTES + 1024;
 
@@ -88,6 +92,7 @@ struct FineParams {
   int g_shift;             // log2(G) when G is a power of two, else -1 (divide)
   long long row0;          // absolute position of chunk row 0
   int box_rows;            // 4 or 8: candidates arrive by TMA boxes of that many key rows; 0: cp.async
+  int box3d;               // box_rows 8: one 3-D box carries both K halves
   uint64_t wait_limit_ns;
 };
 
@@ -154,9 +159,31 @@ __device__ __forceinline__ void f_record(const FineParams& p, volatile int* abor
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_inflight() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(F_IN_FLIGHT - 1) : "memory");
+// The barrier receives one arrival when every cp.async this thread has issued
+// so far has landed (its expected count includes that arrival).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// 3-D TMA tile load (no multicast) at coordinates (x, y, z), completing its
+// bytes on the mbarrier.
+__device__ __forceinline__ void tma_load_3d(void* dst, const void* tmap, uint64_t* bar, int32_t x, int32_t y,
+                                            int32_t z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+// K-major, 128-byte-swizzled operand descriptor with `sbo` bytes between
+// 8-row groups (the layout fields as in sdesc_kmajor_sw128).
+__device__ __forceinline__ uint64_t sdesc_kmajor_sw128_sbo(uint32_t saddr, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(1u) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  d |= static_cast<uint64_t>(2u) << 61;
+  return d;
 }
 __device__ __forceinline__ void cp_async_wait_0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void fence_proxy_async() {
@@ -283,25 +310,27 @@ __global__ void __launch_bounds__(F_THREADS, 1)
             stop = true;
             break;
           }
-          for (int h = 0; h < 2; ++h) {
-            if (!mbar_wait_bounded(&C->full[stage], phase, abort, p.wait_limit_ns)) {
-              f_record(p, abort, FERR_FULL);
-              stop = true;
-              break;
-            }
-            tc_fence_after();
+          if (!mbar_wait_bounded(&C->full[stage], phase, abort, p.wait_limit_ns)) {
+            f_record(p, abort, FERR_FULL);
+            stop = true;
+            break;
+          }
+          tc_fence_after();
+          fence_proxy_async();  // the cp.async path writes through the generic proxy
+          {
             const uint32_t st_addr = a_addr + stage * F_STAGE_BYTES;
 #pragma unroll
-            for (int j = 0; j < F_QT; ++j) {
+            for (int h = 0; h < 2; ++h)
 #pragma unroll
-              for (int kk = 0; kk < 4; ++kk) {
-                const uint32_t kb = kk * 32;  // 16 bf16 of K inside the 128-byte swizzled row
-                mma_bf16(tmem + acc * (F_QT * F_HEADS) + j * F_HEADS,
-                         sdesc_kmajor_sw128(st_addr + j * F_A_QUERY + kb),
-                         sdesc_kmajor_sw128(q_addr + h * F_Q_HALF + j * (F_HEADS * 128) + kb), IDESC,
-                         (h | kk) != 0);
-              }
-            }
+              for (int j = 0; j < F_QT; ++j)
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                  const uint32_t kb = kk * 32;  // 16 bf16 of K inside the 128-byte swizzled row
+                  mma_bf16(tmem + acc * (F_QT * F_HEADS) + j * F_HEADS,
+                           sdesc_kmajor_sw128_sbo(st_addr + j * F_A_QUERY + h * 1024 + kb, F_GROUP),
+                           sdesc_kmajor_sw128(q_addr + h * F_Q_HALF + j * (F_HEADS * 128) + kb), IDESC,
+                           (h | kk) != 0);
+                }
             mma_commit(&C->empty[stage]);
             if (++stage == F_STAGES) {
               stage = 0;
@@ -325,13 +354,14 @@ __global__ void __launch_bounds__(F_THREADS, 1)
     // Every group of 8 candidate slots is 8 consecutive key rows that start
     // on a multiple of gcd(G, 8): a kept block's keys (or 8 of them) or the
     // incomplete block's.  Warp 2, lane l, loads group l % 16 of query l / 16
-    // as 8 / box_rows TMA boxes of box_rows rows x 64 dims per K half (one
-    // 1 KB, 128-byte-swizzled atom of the stage); lane 0 owns the barriers.
+    // into its 2 KB of the stage: with box_rows 8 as one 3-D box (8 rows x
+    // both 64-dim K halves), with box_rows 4 as four 2-D boxes (4 rows x 64
+    // dims); lane 0 owns the barriers.
     // Slots past the row's candidates read key row 0 (their scores are never
     // stored), rows past the keys read as zero.  Warp 3 has nothing to do.
     if (warp == 2) {
       const bool j1 = (lane >> 4) != 0;  // this lane's query, chosen without a dynamic index
-      const int bb = lane & 15, nsub = 8 / p.box_rows;
+      const int bb = lane & 15;
       uint32_t stage = 0, phase = 0;
       uint32_t any_load = 0, last_par = 0;  // per stage: loaded at all / parity of the last load
       bool stop = false;
@@ -356,29 +386,38 @@ __global__ void __launch_bounds__(F_THREADS, 1)
             }
             row[x] = kr;
           }
-          for (int h = 0; h < 2; ++h) {
-            bool got = true;
-            if (lane == 0) {
-              got = mbar_wait_bounded(&C->empty[stage], phase ^ 1u, abort, p.wait_limit_ns);
-              if (!got)
-                f_record(p, abort, FERR_EMPTY);
-              else
-                mbar_arrive_expect_tx(&C->full[stage], F_STAGE_BYTES);
+          bool got = true;
+          if (lane == 0) {
+            got = mbar_wait_bounded(&C->empty[stage], phase ^ 1u, abort, p.wait_limit_ns);
+            if (!got)
+              f_record(p, abort, FERR_EMPTY);
+            else
+              mbar_arrive_expect_tx(&C->full[stage], F_STAGE_BYTES);
+          }
+          if (__shfl_sync(0xFFFFFFFFu, got ? 1 : 0, 0) == 0) {  // the warp gives up as one
+            stop = true;
+            break;
+          }
+          __syncwarp();
+          uint8_t* dst = a_s + stage * F_STAGE_BYTES + (j1 ? F_A_QUERY : 0) + bb * F_GROUP;
+          if (p.box3d) {
+            // both K halves of the 8 rows in one box: [half][row][64 dims]
+            tma_load_3d(dst, &tm_kc, &C->full[stage], 0, row[0], 0);
+          } else if (p.box_rows == 8) {
+            tma_load_2d(dst, &tm_kc, &C->full[stage], 0, row[0]);
+            tma_load_2d(dst + 1024, &tm_kc, &C->full[stage], 64, row[0]);
+          } else {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              tma_load_2d(dst + h * 1024, &tm_kc, &C->full[stage], h * 64, row[0]);
+              tma_load_2d(dst + h * 1024 + 512, &tm_kc, &C->full[stage], h * 64, row[1]);
             }
-            if (__shfl_sync(0xFFFFFFFFu, got ? 1 : 0, 0) == 0) {  // the warp gives up as one
-              stop = true;
-              break;
-            }
-            __syncwarp();
-            uint8_t* dst = a_s + stage * F_STAGE_BYTES + (j1 ? F_A_QUERY : 0) + bb * 1024;
-            tma_load_2d(dst, &tm_kc, &C->full[stage], h * 64, row[0]);
-            if (nsub == 2) tma_load_2d(dst + 512, &tm_kc, &C->full[stage], h * 64, row[1]);
-            any_load |= 1u << stage;
-            last_par = (last_par & ~(1u << stage)) | (phase << stage);
-            if (++stage == F_STAGES) {
-              stage = 0;
-              phase ^= 1u;
-            }
+          }
+          any_load |= 1u << stage;
+          last_par = (last_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == F_STAGES) {
+            stage = 0;
+            phase ^= 1u;
           }
         }
       }
@@ -390,15 +429,15 @@ __global__ void __launch_bounds__(F_THREADS, 1)
     }
   } else if (warp < 4) {
     // ------------------------------------------------------------ gather producers
-    // Thread pt moves 16-byte chunk (pt & 7) of rows (pt >> 3) + 8x, x = 0..15,
-    // of each query's 128-row tile: 8 consecutive threads read one 128-byte
-    // half row.  Chunk c of row r lands at r*128 + ((c ^ (r & 7)) << 4): the
-    // 128-byte swizzle the MMA descriptor expects.
+    // Block sizes not divisible by 4.  Thread pt moves 16-byte chunk (pt & 7)
+    // of rows (pt >> 3) + 8x, x = 0..15, of each query's 128-row tile, both K
+    // halves: 8 consecutive threads read one 128-byte half row.  Chunk c of
+    // row r, half h lands in r's group at h*1024 + (r & 7)*128 + ((c ^ (r & 7))
+    // << 4): the 128-byte swizzle the MMA descriptor expects.  Each thread's
+    // copies of a stage arrive on its barrier when they land (noinc).
     const int pt = threadIdx.x - 64;
     const int ch = pt & 7, rb = pt >> 3;
     uint32_t stage = 0, phase = 0;
-    int pend[F_IN_FLIGHT];  // stages copied into but not yet published, oldest first
-    int n_pend = 0;
     bool stop = false;
     for (int i = 0; !stop; ++i) {
       const int u = f_unit_of(i, n_units);
@@ -425,43 +464,30 @@ __global__ void __launch_bounds__(F_THREADS, 1)
             else if (s < c.count) kk = c.tail0 + (s - c.n_blk_keys);
             key[j][x] = kk < 0 ? 0 : kk;  // an empty slot reads key 0; its score is never stored
           }
-        for (int h = 0; h < 2; ++h) {
-          const bool got = mbar_wait_bounded(&C->empty[stage], phase ^ 1u, abort, p.wait_limit_ns);
-          if (!__all_sync(0xFFFFFFFFu, got)) {  // the warp gives up as one
-            if (lane == 0) f_record(p, abort, FERR_EMPTY);
-            stop = true;
-            break;
-          }
-          const uint32_t base = smem_u32(a_s + stage * F_STAGE_BYTES);
+        const bool got = mbar_wait_bounded(&C->empty[stage], phase ^ 1u, abort, p.wait_limit_ns);
+        if (!__all_sync(0xFFFFFFFFu, got)) {  // the warp gives up as one
+          if (lane == 0) f_record(p, abort, FERR_EMPTY);
+          stop = true;
+          break;
+        }
+        const uint32_t base = smem_u32(a_s + stage * F_STAGE_BYTES);
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
 #pragma unroll
           for (int j = 0; j < F_QT; ++j)
 #pragma unroll
-            for (int x = 0; x < 16; ++x) {
-              const int row = rb + 8 * x;
+            for (int x = 0; x < 16; ++x) {  // row rb + 8x is row rb of group x
               const uint8_t* src = p.kc + static_cast<size_t>(key[j][x]) * (F_DIM * 2) + h * 128 + ch * 16;
-              cp_async16(base + j * F_A_QUERY + row * 128 + ((ch ^ (row & 7)) << 4), src);
+              cp_async16(base + j * F_A_QUERY + x * F_GROUP + h * 1024 + rb * 128 + ((ch ^ rb) << 4), src);
             }
-          cp_async_commit();
-          pend[n_pend++] = static_cast<int>(stage);
-          if (n_pend == F_IN_FLIGHT) {
-            // the oldest outstanding stage's copies have landed: publish them
-            cp_async_wait_inflight();
-            fence_proxy_async();
-            mbar_arrive(&C->full[pend[0]]);
-#pragma unroll
-            for (int e = 0; e + 1 < F_IN_FLIGHT; ++e) pend[e] = pend[e + 1];
-            --n_pend;
-          }
-          if (++stage == F_STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
+        cp_async_arrive_noinc(&C->full[stage]);
+        if (++stage == F_STAGES) {
+          stage = 0;
+          phase ^= 1u;
         }
       }
     }
-    cp_async_wait_0();
-    fence_proxy_async();
-    for (int e = 0; e < n_pend; ++e) mbar_arrive(&C->full[pend[e]]);
+    cp_async_wait_0();  // every copy issued has landed before the CTA can exit
   } else {
     // ------------------------------------------------------------ scoring warps
     const int quad = warp & 3;               // TMEM lanes 32*quad .. +31
@@ -740,12 +766,22 @@ si_status launch_two_stage(const void* q, const void* kc, const float* w, int B,
       if (st != SI_OK) break;
       // candidates come in runs of gcd(G, 8) consecutive key rows starting on
       // a multiple of it; runs of 4 or 8 rows load as TMA boxes of the keys
-      const int box_rows = (G % 8 == 0) ? 8 : (G % 4 == 0) ? 4 : 0;
+      // a multiple of 8 loads both K halves of 8 rows as one 3-D box (the keys
+      // seen as [2 halves][T rows][64 dims]) where the driver takes that
+      // layout, else as two 2-D boxes
+      int box_rows = (G % 8 == 0) ? 8 : (G % 4 == 0) ? 4 : 0;
+      int box3d = 0;
       tm_kc = tm_q;  // unused unless box_rows
-      if (box_rows) {
-        st = encode_tmap_2d(&tm_kc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
-                            static_cast<const uint8_t*>(kc) + static_cast<size_t>(b) * T * F_DIM * 2, F_DIM,
-                            static_cast<uint64_t>(T), F_DIM * 2, 64, box_rows);
+      const uint8_t* kcb = static_cast<const uint8_t*>(kc) + static_cast<size_t>(b) * T * F_DIM * 2;
+      if (box_rows == 8) {
+        const uint64_t dims[3] = {64, static_cast<uint64_t>(T), 2};
+        const uint64_t strides[2] = {F_DIM * 2, 128};
+        const uint32_t box[3] = {64, 8, 2};
+        box3d = try_encode_tmap_3d(&tm_kc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kcb, dims, strides, box) ? 1 : 0;
+      }
+      if (box_rows && !box3d) {
+        st = encode_tmap_2d(&tm_kc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kcb, F_DIM, static_cast<uint64_t>(T),
+                            F_DIM * 2, 64, box_rows);
         if (st != SI_OK) break;
       }
       FineParams fp;
@@ -764,6 +800,7 @@ si_status launch_two_stage(const void* q, const void* kc, const float* w, int B,
       fp.g_shift = (G & (G - 1)) == 0 ? __builtin_ctz(static_cast<unsigned>(G)) : -1;
       fp.row0 = c0;
       fp.box_rows = box_rows;
+      fp.box3d = box3d;
       fp.wait_limit_ns = wait_limit_ns;
       const int units = (R + F_QT - 1) / F_QT;
       fine_score_kernel<<<static_cast<unsigned>(std::min(units, n_sm)), F_THREADS, F_SMEM, stream>>>(tm_q, tm_kc, fp);

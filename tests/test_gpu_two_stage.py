@@ -53,6 +53,8 @@ def test_all_blocks_kept_equals_one_stage():
     (1, 4096, 1024, 4, 64, 8, 16, 0),      # 128 blocks, 16 kept
     (2, 1030, 300, 3, 32, 4, 10, 300),     # m = 3, blocks of 4, odd rows, chunks of 300
     (1, 2048, 512, 4, 200, 8, 12, 1000),   # k > 8 * n_keep for late rows: candidates < k
+    (1, 2048, 600, 4, 64, 6, 20, 0),       # blocks of 6: the cp.async gather (no whole TMA boxes)
+    (1, 1024, 520, 2, 96, 16, 9, 0),       # blocks of 16: two 8-row boxes per block
 ])
 def test_integer_two_stage_bit_exact(B, S, T, m, k, G, n_keep, chunk):
     """Integer inputs: pooled keys, coarse and fine scores are exact in fp32,
