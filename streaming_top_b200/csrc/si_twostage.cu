@@ -372,20 +372,27 @@ __global__ void __launch_bounds__(F_THREADS, 1)
         const int rj = j1 ? U.r[1] : U.r[0];
         const Cand c = j1 ? U.c[1] : U.c[0];
         const int32_t* crow = p.coarse + static_cast<size_t>(rj < p.R ? rj : 0) * p.n_keep;
+        // the key rows of this lane's group of tile t (at most two runs of 4):
+        // the kept-block entries of tile t + 1 are loaded (unconditionally,
+        // clamped in range) while tile t's boxes are issued, and turned into
+        // rows one tile later, so their latency is hidden
+        auto load_blk = [&](int t, int* blk) {
+#pragma unroll
+          for (int x = 0; x < 2; ++x) blk[x] = crow[min(blk_slot(p, t * F_KT + 8 * bb + x * 4), p.n_keep - 1)];
+        };
+        int blk_next[2];
+        load_blk(0, blk_next);
         for (int t = 0; t < U.nt && !stop; ++t) {
           int row[2];
 #pragma unroll
           for (int x = 0; x < 2; ++x) {
-            const int s1 = t * F_KT + 8 * bb + x * 4;
+            const int s1 = t * F_KT + 8 * bb + x * 4, blk = blk_next[x];
             int kr = 0;
-            if (s1 < c.n_blk_keys) {
-              const int blk = crow[min(blk_slot(p, s1), p.n_keep - 1)];
-              kr = blk >= 0 && blk < p.nb ? blk * p.G + in_blk(p, s1) : 0;
-            } else if (s1 < c.count) {
-              kr = c.tail0 + (s1 - c.n_blk_keys);
-            }
+            if (s1 < c.n_blk_keys) kr = blk >= 0 && blk < p.nb ? blk * p.G + in_blk(p, s1) : 0;
+            else if (s1 < c.count) kr = c.tail0 + (s1 - c.n_blk_keys);
             row[x] = kr;
           }
+          if (t + 1 < U.nt) load_blk(t + 1, blk_next);
           bool got = true;
           if (lane == 0) {
             got = mbar_wait_bounded(&C->empty[stage], phase ^ 1u, abort, p.wait_limit_ns);
