@@ -91,8 +91,8 @@ struct FineParams {
   int nb;                  // complete blocks of the sequence, T / G
   int g_shift;             // log2(G) when G is a power of two, else -1 (divide)
   long long row0;          // absolute position of chunk row 0
-  int box_rows;            // 4 or 8: candidates arrive by TMA boxes of that many key rows; 0: cp.async
-  int box3d;               // box_rows 8: one 3-D box carries both K halves
+  int box_rows;            // 8 (3-D boxes) or 4 (2-D boxes): candidates arrive by TMA; 0: cp.async
+  int box3d;               // 1 with box_rows 8: one 3-D box carries 8 rows, both K halves
   uint64_t wait_limit_ns;
 };
 
@@ -410,10 +410,7 @@ __global__ void __launch_bounds__(F_THREADS, 1)
           if (p.box3d) {
             // both K halves of the 8 rows in one box: [half][row][64 dims]
             tma_load_3d(dst, &tm_kc, &C->full[stage], 0, row[0], 0);
-          } else if (p.box_rows == 8) {
-            tma_load_2d(dst, &tm_kc, &C->full[stage], 0, row[0]);
-            tma_load_2d(dst + 1024, &tm_kc, &C->full[stage], 64, row[0]);
-          } else {
+          } else {  // box_rows 4: four 2-D boxes of 4 rows x 64 dims
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               tma_load_2d(dst + h * 1024, &tm_kc, &C->full[stage], h * 64, row[0]);
@@ -775,20 +772,21 @@ si_status launch_two_stage(const void* q, const void* kc, const float* w, int B,
       // a multiple of it; runs of 4 or 8 rows load as TMA boxes of the keys
       // a multiple of 8 loads both K halves of 8 rows as one 3-D box (the keys
       // seen as [2 halves][T rows][64 dims]) where the driver takes that
-      // layout, else as two 2-D boxes
-      int box_rows = (G % 8 == 0) ? 8 : (G % 4 == 0) ? 4 : 0;
+      // layout; a multiple of 4 (or a refused 3-D map) as 2-D boxes of 4 rows
+      int box_rows = (G % 4 == 0) ? 4 : 0;
       int box3d = 0;
       tm_kc = tm_q;  // unused unless box_rows
       const uint8_t* kcb = static_cast<const uint8_t*>(kc) + static_cast<size_t>(b) * T * F_DIM * 2;
-      if (box_rows == 8) {
+      if (G % 8 == 0) {
         const uint64_t dims[3] = {64, static_cast<uint64_t>(T), 2};
         const uint64_t strides[2] = {F_DIM * 2, 128};
         const uint32_t box[3] = {64, 8, 2};
         box3d = try_encode_tmap_3d(&tm_kc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kcb, dims, strides, box) ? 1 : 0;
+        if (box3d) box_rows = 8;
       }
-      if (box_rows && !box3d) {
+      if (box_rows == 4) {
         st = encode_tmap_2d(&tm_kc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kcb, F_DIM, static_cast<uint64_t>(T),
-                            F_DIM * 2, 64, box_rows);
+                            F_DIM * 2, 64, 4);
         if (st != SI_OK) break;
       }
       FineParams fp;

@@ -86,6 +86,40 @@ def test_attention_over_the_indexer_selection():
     _check(q, kv, np.ascontiguousarray(sel))
 
 
+def test_attention_full_size_sampled_rows():
+    """The launch the bench times: 65,536 queries x 64 heads over T = 16,384
+    latents, each query's selection the indexer's top-512 of the planted
+    v4flash inputs (seed 3), the attention inputs drawn as the bench draws
+    them.  48 sampled queries (the first, the last, and uniformly drawn ones)
+    against the oracle, the rest only for finiteness."""
+    wl = synth.WORKLOADS["v4flash"]
+    inp = synth.make_inputs(wl)
+    qi = torch.from_numpy(inp["q"].view(np.int16)).view(torch.bfloat16).cuda()
+    kc = torch.from_numpy(inp["kc"].view(np.int16)).view(torch.bfloat16).cuda()
+    idx, _ = si.indexer_topk(qi, kc, torch.from_numpy(inp["w"]).cuda(), wl.m, wl.k)
+    del qi, kc, inp
+    q, kv = synth.attention_inputs(wl.B, wl.S, wl.T, seed=wl.seed + 500)
+    qd = torch.from_numpy(q.view(np.int16)).view(torch.bfloat16).cuda()
+    kd = torch.from_numpy(kv.view(np.int16)).view(torch.bfloat16).cuda()
+    out, lse = si.sparse_attention(qd, kd, idx)
+    assert si.device_status() == si.SI_OK
+    del qd, kd
+    rows = np.unique(np.r_[0, 1, wl.S - 1, synth.sample_rows(45, 2, wl.S - 1, seed=11)])
+    rt = torch.from_numpy(rows).cuda()
+    go = out[:, rt].float().cpu().numpy()
+    gl = lse[:, rt].cpu().numpy()
+    sel = np.ascontiguousarray(idx[:, rt].cpu().numpy())
+    ro, rl = oracle.sparse_attention(np.ascontiguousarray(q[:, rows]), kv, sel, DV)
+    vmax = np.abs(_bf16_to_f32(kv[..., :DV])).max()
+    err = np.abs(go - ro)
+    assert np.all(err <= 2.0 ** -8 * vmax + 2.0 ** -9 * np.abs(ro)), float(err.max())
+    fin = np.isfinite(rl)
+    assert np.array_equal(fin, np.isfinite(gl)) and np.all(np.isneginf(gl[~fin]))
+    assert np.all(np.abs(gl[fin] - rl[fin]) <= 4e-3), float(np.abs(gl[fin] - rl[fin]).max())
+    # every query attends over at least one key (query t sees (t+1)//4 >= 1 keys from t = 3 on)
+    assert bool(torch.isfinite(lse[:, 3:]).all())
+
+
 def test_attention_special_cases():
     T, k = 256, 128
     q, kv = synth.attention_inputs(1, 4, T, seed=9)
