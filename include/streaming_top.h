@@ -239,6 +239,10 @@ SI_API si_status si_indexer_materialize_noalloc(const void* q, const void* kc, c
  * chunks of opt->query_chunk rows (0 = 16384); scratch of
  * si_two_stage_workspace_size() bytes comes from opt->workspace when given,
  * else it is allocated and freed on `stream`.  Asynchronous on `stream`.
+ * Performance: a block size divisible by 8 (the notes' 8) loads each 8-key
+ * run of candidates as one TMA box; one divisible by 4 as two smaller ones;
+ * other sizes gather the candidate rows 16 bytes at a time, several times
+ * slower.  kc must be 16-byte aligned (as for si_indexer_topk).
  */
 SI_API si_status si_indexer_topk_two_stage(const void* q, const void* kc, const float* w, int B, int S, int T,
                                            int H_I, int D, int m, int k, int block, int n_keep,
