@@ -559,12 +559,90 @@ __global__ void __launch_bounds__(F_THREADS, 1)
 
 // ---------------------------------------------------------------- select
 // Exact top-k of a row's packed candidate keys (distinct: the low half is
-// ~index): radix select of the k-th largest key, 8 bits a pass from the
-// top, with per-warp histograms fed by warp-aggregated atomics; a pass whose
-// boundary bin is taken whole ends the search.  The k keys >= the threshold
-// are stored in no particular order (the row sort orders them).
+// ~index).  A first pass bins the keys by where their orderable score falls in
+// the row's own range (2048 bins, shared-memory atomics) and finds the bin B
+// that holds the k-th largest; the keys above B are in.  When B is not taken
+// whole, its keys (usually a handful) go to a list and a radix select (8 bits
+// a pass from the top, per-warp histograms fed by warp-aggregated atomics)
+// picks the ones still needed; a bin of more than S_LCAP keys (many equal
+// scores) falls back to the radix select over the whole row.  The k keys are
+// stored in no particular order (the row sort orders them).
 constexpr int S_THREADS = 512;
 constexpr int S_WARPS = S_THREADS / 32;
+constexpr int S_BINS = 2048;   // first-pass bins, 4 a thread
+constexpr int S_LCAP = 4096;   // largest boundary bin handled as a list
+static_assert(S_BINS == 4 * S_THREADS, "the bin scan gives each thread 4 bins");
+
+// Block-wide: the largest prefix p such that at least `need` of keys[0..cnt)
+// are >= p, built 8 bits a pass from the top (the threshold of the need-th
+// largest key).  `hist` is [S_WARPS][256], `tot` [256].
+__device__ uint64_t radix_threshold(const uint64_t* keys, int cnt, uint32_t need, uint32_t* hist, uint32_t* tot,
+                                    uint64_t* s_prefix, uint32_t* s_need, uint32_t* s_done) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  __syncthreads();  // the caller's shared state is settled
+  if (tid == 0) {
+    *s_prefix = 0;
+    *s_need = need;
+    *s_done = static_cast<uint32_t>(cnt) <= need ? 1u : 0u;
+  }
+  __syncthreads();
+  uint64_t mask = 0;
+  for (int shift = 56; shift >= 0 && !*s_done; shift -= 8) {
+    for (int i = tid; i < S_WARPS * 256; i += S_THREADS) hist[i] = 0;
+    __syncthreads();
+    const uint64_t prefix = *s_prefix;
+    for (int i0 = 0; i0 < cnt; i0 += S_THREADS) {
+      const int i = i0 + tid;
+      const bool in = i < cnt && (keys[i < cnt ? i : 0] & mask) == prefix;
+      const uint32_t d = in ? static_cast<uint32_t>(keys[i] >> shift) & 255u : 256u;
+      const uint32_t peers = __match_any_sync(0xFFFFFFFFu, d);
+      if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[warp * 256 + d], __popc(peers));
+    }
+    __syncthreads();
+    if (tid < 256) {
+      uint32_t sum = 0;
+      for (int w = 0; w < S_WARPS; ++w) sum += hist[w * 256 + tid];
+      tot[tid] = sum;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      // lane l holds bins 255-8l .. 248-8l; find the bin where the count
+      // from the top reaches `need`
+      uint32_t v[8], sum = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        v[e] = tot[255 - 8 * lane - e];
+        sum += v[e];
+      }
+      uint32_t incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const uint32_t nd = *s_need, excl = incl - sum;
+      if (excl < nd && nd <= incl) {
+        uint32_t above = excl;
+        int b = 0;
+        for (int e = 0; e < 8; ++e) {
+          if (above + v[e] >= nd) {
+            b = 255 - 8 * lane - e;
+            break;
+          }
+          above += v[e];
+        }
+        *s_prefix = prefix | (static_cast<uint64_t>(b) << shift);
+        *s_need = nd - above;
+        if (nd - above == tot[b]) *s_done = 1u;  // the whole bin is in: threshold found
+      }
+    }
+    mask |= static_cast<uint64_t>(255) << shift;
+    __syncthreads();
+  }
+  const uint64_t thr = *s_prefix;
+  __syncthreads();  // every thread has read the threshold
+  return thr;
+}
 
 __global__ void __launch_bounds__(S_THREADS) select_topk_kernel(const uint64_t* __restrict__ packed,
                                                                 const FineParams p, int k, int32_t* out_idx,
@@ -572,9 +650,12 @@ __global__ void __launch_bounds__(S_THREADS) select_topk_kernel(const uint64_t* 
   extern __shared__ __align__(16) uint8_t s_raw[];
   uint32_t* hist = reinterpret_cast<uint32_t*>(s_raw);          // [S_WARPS][256]
   uint32_t* tot = hist + S_WARPS * 256;                          // [256]
-  uint64_t* keys = reinterpret_cast<uint64_t*>(tot + 256 + 4);   // [ldp]
+  uint32_t* bins = tot + 256 + 4;                                // [S_BINS]
+  uint64_t* list = reinterpret_cast<uint64_t*>(bins + S_BINS);   // [S_LCAP]
+  uint64_t* keys = list + S_LCAP;                                // [ldp]
   __shared__ uint64_t s_prefix;
-  __shared__ uint32_t s_need, s_done, s_out;
+  __shared__ uint32_t s_need, s_done, s_out, s_nl, s_B, s_A, s_cB;
+  __shared__ uint32_t s_max[S_WARPS], s_min[S_WARPS], s_wsum[S_WARPS];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   for (int r = blockIdx.x; r < p.R; r += gridDim.x) {
     const Cand c = cand_of(p, r);
@@ -582,73 +663,104 @@ __global__ void __launch_bounds__(S_THREADS) select_topk_kernel(const uint64_t* 
     const uint64_t* row = packed + static_cast<size_t>(r) * p.ldp;
     int32_t* oi = out_idx + static_cast<size_t>(r) * k;
     float* os = out_score + static_cast<size_t>(r) * k;
-    for (int i = tid; i < cnt; i += S_THREADS) keys[i] = row[i];
+    // keys into shared memory, and the range of their orderable scores
+    uint32_t mx = 0u, mn = 0xFFFFFFFFu;
+    for (int i = tid; i < cnt; i += S_THREADS) {
+      const uint64_t x = row[i];
+      keys[i] = x;
+      const uint32_t hi = static_cast<uint32_t>(x >> 32);
+      mx = max(mx, hi);
+      mn = min(mn, hi);
+    }
+    for (int i = tid; i < S_BINS; i += S_THREADS) bins[i] = 0u;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+      mn = min(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, o));
+    }
+    if (lane == 0) {
+      s_max[warp] = mx;
+      s_min[warp] = mn;
+    }
     if (tid == 0) {
-      s_prefix = 0;
-      s_need = static_cast<uint32_t>(k);
-      s_done = cnt <= k ? 1u : 0u;
       s_out = 0;
+      s_nl = 0;
     }
     __syncthreads();
-    uint64_t mask = 0;
-    for (int shift = 56; shift >= 0 && !s_done; shift -= 8) {
-      for (int i = tid; i < S_WARPS * 256; i += S_THREADS) hist[i] = 0;
-      __syncthreads();
-      const uint64_t prefix = s_prefix;
-      for (int i0 = 0; i0 < cnt; i0 += S_THREADS) {
-        const int i = i0 + tid;
-        const bool in = i < cnt && (keys[i < cnt ? i : 0] & mask) == prefix;
-        const uint32_t d = in ? static_cast<uint32_t>(keys[i] >> shift) & 255u : 256u;
-        const uint32_t peers = __match_any_sync(0xFFFFFFFFu, d);
-        if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[warp * 256 + d], __popc(peers));
-      }
-      __syncthreads();
-      if (tid < 256) {
-        uint32_t s = 0;
-        for (int w = 0; w < S_WARPS; ++w) s += hist[w * 256 + tid];
-        tot[tid] = s;
-      }
-      __syncthreads();
-      if (warp == 0) {
-        // lane l holds bins 255-8l .. 248-8l; find the bin where the count
-        // from the top reaches `need`
-        uint32_t v[8], sum = 0;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          v[e] = tot[255 - 8 * lane - e];
-          sum += v[e];
-        }
-        uint32_t incl = sum;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-          if (lane >= o) incl += y;
-        }
-        const uint32_t need = s_need, excl = incl - sum;
-        const bool mine = excl < need && need <= incl;
-        if (mine) {
-          uint32_t above = excl;
-          int b = 0;
-          for (int e = 0; e < 8; ++e) {
-            if (above + v[e] >= need) {
-              b = 255 - 8 * lane - e;
-              break;
-            }
-            above += v[e];
-          }
-          s_prefix = prefix | (static_cast<uint64_t>(b) << shift);
-          s_need = need - above;
-          if (need - above == tot[b]) s_done = 1u;  // the whole bin is in: threshold found
-        }
-      }
-      mask |= static_cast<uint64_t>(255) << shift;
-      __syncthreads();
+    for (int w = 0; w < S_WARPS; ++w) {
+      mx = max(mx, s_max[w]);
+      mn = min(mn, s_min[w]);
     }
-    // keys >= threshold: exactly min(k, cnt) of them
-    const uint64_t thr = cnt <= k ? 0ull : s_prefix;
+    // modes: 0 take all, 1 bins <= B, 2 bins < B plus the list's best, 3 keys >= thr
+    int mode = 0, B = 0, sh = 0;
+    uint64_t thr = 0ull;
+    if (cnt > k) {
+      const uint32_t range = mx - mn;
+      const int bl = range ? 32 - __clz(static_cast<int>(range)) : 0;
+      sh = bl > 11 ? bl - 11 : 0;
+      for (int i = tid; i < cnt; i += S_THREADS)
+        atomicAdd(&bins[(mx - static_cast<uint32_t>(keys[i] >> 32)) >> sh], 1u);
+      __syncthreads();
+      // exclusive scan of the bins from the top: thread t owns bins 4t .. 4t+3
+      uint32_t cb[4], sum = 0u;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        cb[e] = bins[4 * tid + e];
+        sum += cb[e];
+      }
+      uint32_t incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (lane == 31) s_wsum[warp] = incl;
+      __syncthreads();
+      uint32_t excl = incl - sum;
+      for (int w = 0; w < warp; ++w) excl += s_wsum[w];
+      const uint32_t kk = static_cast<uint32_t>(k);
+      if (excl < kk && kk <= excl + sum) {
+        uint32_t above = excl;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if (above + cb[e] >= kk) {
+            s_B = 4 * tid + e;
+            s_A = above;
+            s_cB = cb[e];
+            break;
+          }
+          above += cb[e];
+        }
+      }
+      __syncthreads();
+      B = static_cast<int>(s_B);
+      const uint32_t need = kk - s_A, cB = s_cB;
+      if (need == cB) {
+        mode = 1;
+      } else if (cB <= static_cast<uint32_t>(S_LCAP)) {
+        for (int i = tid; i < cnt; i += S_THREADS) {
+          const uint64_t x = keys[i];
+          if (static_cast<int>((mx - static_cast<uint32_t>(x >> 32)) >> sh) == B) list[atomicAdd(&s_nl, 1u)] = x;
+        }
+        thr = radix_threshold(list, static_cast<int>(cB), need, hist, tot, &s_prefix, &s_need, &s_done);
+        mode = 2;
+      } else {
+        thr = radix_threshold(keys, cnt, kk, hist, tot, &s_prefix, &s_need, &s_done);
+        mode = 3;
+      }
+    }
+    // the chosen keys: exactly min(k, cnt) of them
     for (int i0 = 0; i0 < cnt; i0 += S_THREADS) {
       const int i = i0 + tid;
-      const bool take = i < cnt && keys[i < cnt ? i : 0] >= thr;
+      bool take = false;
+      uint64_t x = 0ull;
+      if (i < cnt) {
+        x = keys[i];
+        const int b = static_cast<int>((mx - static_cast<uint32_t>(x >> 32)) >> sh);
+        take = mode == 0 || (mode == 1 && b <= B) || (mode == 2 && (b < B || (b == B && x >= thr))) ||
+               (mode == 3 && x >= thr);
+      }
       const uint32_t bal = __ballot_sync(0xFFFFFFFFu, take);
       uint32_t base = 0;
       if (lane == 0 && bal) base = atomicAdd(&s_out, __popc(bal));
@@ -656,7 +768,6 @@ __global__ void __launch_bounds__(S_THREADS) select_topk_kernel(const uint64_t* 
       if (take) {
         const uint32_t pos = base + __popc(bal & ((1u << lane) - 1u));
         if (pos < static_cast<uint32_t>(k)) {
-          const uint64_t x = keys[i];
           const uint32_t o = static_cast<uint32_t>(x >> 32);
           oi[pos] = static_cast<int32_t>(~static_cast<uint32_t>(x));
           os[pos] = __uint_as_float((o & 0x80000000u) ? (o & 0x7FFFFFFFu) : ~o);
@@ -726,7 +837,8 @@ si_status launch_two_stage(const void* q, const void* kc, const float* w, int B,
     e = cudaFuncSetAttribute(fine_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, F_SMEM);
     if (e != cudaSuccess) st = cuda_fail(e, "cudaFuncSetAttribute(fine_score_kernel)");
   }
-  const size_t sel_smem = static_cast<size_t>(S_WARPS) * 256 * 4 + 256 * 4 + 16 + static_cast<size_t>(ldp) * 8;
+  const size_t sel_smem = static_cast<size_t>(S_WARPS) * 256 * 4 + 256 * 4 + 16 + S_BINS * 4 +
+                          static_cast<size_t>(S_LCAP) * 8 + static_cast<size_t>(ldp) * 8;
   if (st == SI_OK) {
     e = cudaFuncSetAttribute(select_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(sel_smem));
