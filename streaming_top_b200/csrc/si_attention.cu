@@ -12,22 +12,24 @@
 //
 // One CTA per SM, persistent over queries.  Per query:
 //   QK   S^T[e, h] = sum_d kv[sel[e], d] * q[h, d]: tcgen05 kind::f16, A = 128
-//        gathered latent rows (M = entries) x 64 dims per stage (TMA gather4),
-//        SW128 K-major; B = q[t] (N = 64 heads, K = 576) TMA-loaded once; fp32 into
+//        gathered latent rows (M = entries) x 64 dims per 16 KB stage, SW128
+//        K-major; B = q[t] (N = 64 heads, K = 576) TMA-loaded once; fp32 into
 //        TMEM columns [64 j, 64 j + 64) for entry tile j.
-//   soft max and sum per head over the k entries (4 softmax warps, lane =
-//        entry, 32 heads at a time), P = exp(scale (s - max)) rounded to bf16
-//        and written as P^T (N = heads, K = entries, SW128 K-major), the sums
-//        of the rounded P kept for the normalisation, lse = scale max + ln sum.
-//   PV   O^T[dv, h] = sum_e V[e, dv] P^T[h, e]: A = gathered value tiles read
-//        MN-major (M = dv, contiguous in each latent row; 128 dv x 64 entries
-//        per stage), B = P^T; fp32 into TMEM columns [256 + 64 v, ...) for dv
-//        tile v.
+//   softmax over the k entries per head (4 warps, lane = entry): (1) the max,
+//        (2) tile by tile P = exp(scale (s - max)) rounded to bf16 and written
+//        as P^T (N = heads, K = entries, SW128 K-major), each tile released to
+//        the MMA warp by its own barrier, (3) the sums of the rounded P for the
+//        normalisation and lse = scale max + ln sum.
+//   PV   O^T[dv, h] = sum_e V[e, dv] P^T[h, e], chunk by chunk (64 entries, the
+//        four 128-dv tiles): A = gathered value tiles read MN-major (dv is
+//        contiguous in each latent row), B = P^T; fp32 into TMEM columns
+//        [256 + 64 v, ...) for dv tile v.
 //   out  O[t, h, dv] = O^T * (1 / sum_h), bf16; lse[t, h] fp32.
-// Warps: 0 q loads (TMA), 1 MMA issue, 2-3 gather producers (half of each
-// stage by TMA gather4, half by 16-byte cp.async), 4-7 softmax and epilogue.  Every wait
-// is bounded; on expiry the kernel records SI_ERR_TIMEOUT, drains its copies
-// and MMAs and exits.
+// Warps: 0 q loads (TMA), 1 MMA issue, 2-3 gather producers (each stage half
+// by TMA gather4 from warp 2, half by 16-byte cp.async from warp 3: the two
+// copy paths' rates add up), 4-7 softmax and epilogue.  Every wait is bounded;
+// on expiry the kernel records SI_ERR_TIMEOUT, drains its copies and MMAs and
+// exits.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
