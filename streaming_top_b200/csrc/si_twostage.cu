@@ -15,17 +15,19 @@
 //             compression m*G (block j is complete for query t iff
 //             j*(m*G) + m*G - 1 <= t: the same visibility rule) and k = n_keep,
 //             rows left unsorted -- a query's kept blocks.
-//   fine    : this file's tcgen05 kernel.  A work unit is 2 queries; for
-//             each 128-candidate tile, producer warps gather every query's
-//             candidate key rows with cp.async straight into the 128-byte-
-//             swizzled K-major layout the MMA reads (two K halves per tile,
-//             6 stages, 4 copy groups in flight), one thread issues M = 128 keys x N = 64
-//             heads MMAs per query into a TMEM double buffer, and 8 scoring
-//             warps apply ReLU and the head weights and store each
-//             candidate's packed key (orderable score << 32 | ~index).
-//   select  : an exact radix select of the k largest packed keys per row
-//             (8-bit digits, warp-aggregated shared-memory histograms), then
-//             the row sort orders them.
+//   fine    : this file's tcgen05 kernel.  A work unit is 2 queries; each
+//             128-candidate tile (both queries, both 64-dim K halves, 64 KB, 3
+//             stages) arrives in the 128-byte-swizzled K-major layout the MMA
+//             reads: for block sizes divisible by 8 one 3-D TMA box per run of
+//             8 key rows, by 4 four 2-D boxes, otherwise 16-byte cp.async.
+//             One thread issues M = 128 keys x N = 64 heads MMAs per query
+//             into a TMEM double buffer, and 8 scoring warps apply ReLU and
+//             the head weights and store each candidate's packed key
+//             (orderable score << 32 | ~index).
+//   select  : the exact k largest packed keys per row: one pass over 2048
+//             bins of the row's score range, a radix select (8-bit digits,
+//             warp-aggregated shared-memory histograms) inside the boundary
+//             bin; then the row sort orders them.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
